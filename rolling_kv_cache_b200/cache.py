@@ -1,0 +1,168 @@
+"""User-facing Python API over the C ABI.
+
+``RollingKVCache`` owns one rc handle and its device memory block (a torch
+uint8 tensor; torch is used only for memory and streams). ``step`` runs one
+chunk through one layer in the library's kernels; it accepts device tensors,
+or host tensors (pinned for speed), in which case it copies them to the
+device, runs the step and copies the output back.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import binding as B
+
+
+def make_config(*, layers: int, heads: int, head_dim: int, grid_h: int, grid_w: int,
+                sink_frames: int, window_frames: int, chunk_frames: int = 3,
+                policy: int = B.RC_SLIDING, mask_block_frames: int = 1, theta: float = 10000.0,
+                t_max: int = 4096, rope_pairs=(0, 0, 0), rs_bank_blocks: int = 0,
+                rs_sink_blocks: int = 0, rs_static_semantics: int = 0, ir_f_limit: int = 0,
+                ir_sink_blocks: int = 0, ir_cache_blocks: int = 0) -> B.rc_config:
+    cfg = B.rc_config_init(layers, heads, head_dim, grid_h * grid_w, sink_frames, window_frames)
+    cfg.grid_h, cfg.grid_w = grid_h, grid_w
+    cfg.chunk_frames = chunk_frames
+    cfg.policy = policy
+    cfg.mask_block_frames = mask_block_frames
+    cfg.theta = theta
+    cfg.t_max = t_max
+    cfg.rope_t_pairs, cfg.rope_h_pairs, cfg.rope_w_pairs = rope_pairs
+    cfg.rs_bank_blocks, cfg.rs_sink_blocks = rs_bank_blocks, rs_sink_blocks
+    cfg.rs_static_semantics = rs_static_semantics
+    cfg.ir_f_limit, cfg.ir_sink_blocks, cfg.ir_cache_blocks = ir_f_limit, ir_sink_blocks, ir_cache_blocks
+    return cfg
+
+
+class RollingKVCache:
+    """Bounded KV cache of every layer of one video stream.
+
+    device=None creates a host-only handle (integer state only, no GPU).
+    """
+
+    def __init__(self, cfg: B.rc_config, device: Optional[torch.device] = torch.device("cuda")):
+        self.cfg = cfg
+        self.nbytes = B.rc_cache_bytes(cfg)
+        self.device = device
+        self.mem = None
+        ptr = 0
+        if device is not None:
+            if not torch.cuda.is_available():
+                raise RuntimeError("a device cache needs CUDA")
+            self.mem = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
+            ptr = (self.mem.data_ptr() + 255) // 256 * 256
+        self.handle = B.rc_cache_create(cfg, ptr, self.nbytes)
+        self._staging = {}
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            B.rc_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):  # pragma: no cover
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def policy(self) -> int:
+        return self.cfg.policy
+
+    def _stream(self) -> int:
+        return torch.cuda.current_stream(self.device).cuda_stream if self.device is not None else 0
+
+    def step(self, layer: int, q, k, v, frame_start: int, out=None, lse=None, scores=None,
+             topc=None, C: int = 0):
+        """One chunk through one layer. q/k/v: [n_frames*F, H, d] bf16.
+
+        Host-only handles take q=k=v=None and only advance the state.
+        Returns ``out`` ([n_frames*F, H, d] bf16).
+        """
+        F = self.cfg.frame_seqlen
+        if self.device is None:
+            B.rc_step(self.handle, layer, 0, 0, 0, frame_start, self._n_frames(q, frame_start),
+                      self.cfg.policy, 0)
+            return None
+        host = not q.is_cuda
+        if host:
+            q = q.to(self.device, non_blocking=True)
+            k = k.to(self.device, non_blocking=True)
+            v = v.to(self.device, non_blocking=True)
+        for t in (q, k, v):
+            if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 3:
+                raise ValueError("q/k/v must be contiguous [n_tok, H, d] bf16")
+        n_tok = q.shape[0]
+        if n_tok % F:
+            raise ValueError("token count must be whole frames")
+        if out is None or host:
+            out_dev = torch.empty_like(q)
+        else:
+            out_dev = out
+        B.rc_step(self.handle, layer, q.data_ptr(), k.data_ptr(), v.data_ptr(), frame_start,
+                  n_tok // F, self.cfg.policy, out_dev.data_ptr(),
+                  lse.data_ptr() if lse is not None else 0,
+                  scores.data_ptr() if scores is not None else 0,
+                  topc.data_ptr() if topc is not None else 0, C, self._stream())
+        if host:
+            if out is None:
+                out = torch.empty(out_dev.shape, dtype=out_dev.dtype, pin_memory=True)
+            out.copy_(out_dev, non_blocking=True)
+            return out
+        return out_dev
+
+    def _n_frames(self, q, frame_start):
+        return self.cfg.chunk_frames if q is None else q.shape[0] // self.cfg.frame_seqlen
+
+    def reindex(self, t_delta: int, flags: int) -> None:
+        B.rc_reindex(self.handle, self.cfg.policy, t_delta, flags, 0)
+
+    def state(self, layer: int = 0) -> B.rc_state:
+        return B.rc_get_state(self.handle, layer)
+
+    def kept(self, layer: int = 0):
+        """[(content, tau, region, rank, slot, stored_time)] in logical order."""
+        st = self.state(layer)
+        return [(e.content, e.tau, e.region, e.rank, e.slot, e.stored_time)
+                for e in st.kept[:st.n_kept]]
+
+    def device_status(self) -> None:
+        B.rc_device_status(self.handle, self._stream())
+
+    def _region(self, offset: int, nbytes: int) -> torch.Tensor:
+        base = (self.mem.data_ptr() + 255) // 256 * 256 - self.mem.data_ptr()
+        return self.mem[base + offset: base + offset + nbytes]
+
+    def cache_views(self, layer: int):
+        """(K, V) torch views [H, capacity, d] bf16 of one layer's ring buffers."""
+        if self.mem is None:
+            raise RuntimeError("host-only handle")
+        lay = B.rc_cache_layout(self.handle)
+        H, d = self.cfg.heads, self.cfg.head_dim
+        n = H * lay.capacity * d * 2
+        o = layer * lay.kv_layer_stride
+        k = self._region(lay.k_offset + o, n).view(torch.bfloat16).view(H, lay.capacity, d)
+        v = self._region(lay.v_offset + o, n).view(torch.bfloat16).view(H, lay.capacity, d)
+        return k, v
+
+    def raw_views(self, layer: int):
+        """(raw K, raw V or None) views [H, raw_frames*F, d] of the pristine source."""
+        lay = B.rc_cache_layout(self.handle)
+        H, d, F = self.cfg.heads, self.cfg.head_dim, self.cfg.frame_seqlen
+        n = H * lay.raw_frames * F * d * 2
+        o = layer * lay.raw_layer_stride
+        rk = self._region(lay.raw_k_offset + o, n).view(torch.bfloat16).view(H, -1, d) if lay.raw_k_offset else None
+        rv = self._region(lay.raw_v_offset + o, n).view(torch.bfloat16).view(H, -1, d) if lay.raw_v_offset else None
+        return rk, rv
+
+    def q_rot_view(self, n_tok: int):
+        """Rotated queries [H, n_tok, d] of the last step (scratch; valid until the next step)."""
+        lay = B.rc_cache_layout(self.handle)
+        H, d = self.cfg.heads, self.cfg.head_dim
+        stride = self.cfg.chunk_frames * self.cfg.frame_seqlen
+        full = self._region(lay.q_offset, H * stride * d * 2).view(torch.bfloat16).view(H, stride, d)
+        return full[:, :n_tok]
+
+    def watchdog_selftest(self, limit_us: int = 20000) -> None:
+        B.rc_watchdog_selftest(self.handle, limit_us, self._stream())

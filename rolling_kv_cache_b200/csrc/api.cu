@@ -1,0 +1,483 @@
+// C ABI (include/rc.h): memory plan, RoPE tables, TMA descriptors and the
+// launch sequence of one step. Host code; kernels live in the other .cu files.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <memory>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/rc.h"
+#include "engine.hpp"
+#include "kernels.cuh"
+
+namespace {
+
+thread_local std::string g_err;
+
+rc_status set_err(rc_status st, const std::string& m) {
+  g_err = m;
+  return st;
+}
+
+rc_status cuda_err(cudaError_t e, const char* what) {
+  return set_err(RC_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct MemPlan {
+  size_t kv_bytes, raw_bytes, q_bytes, lse_bytes, score_bytes, tab_t, tab_h, tab_w, status_bytes;
+  size_t off_kv, off_raw, off_q, off_lse, off_score_phys, off_score_logical, off_tab_t, off_tab_h,
+      off_tab_w, off_status, total;
+  int pt, ph, pw, cap, raw_frames, q_stride;
+};
+
+MemPlan plan_memory(const rc_config& c, int raw_frames) {
+  MemPlan m{};
+  m.pt = c.rope_t_pairs;
+  m.ph = c.rope_h_pairs;
+  m.pw = c.rope_w_pairs;
+  if (m.pt == 0 && m.ph == 0 && m.pw == 0) rc::DefaultPairs(c.head_dim, &m.pt, &m.ph, &m.pw);
+  m.cap = (c.sink_frames + c.window_frames) * c.frame_seqlen;
+  m.raw_frames = raw_frames;
+  m.q_stride = c.chunk_frames * c.frame_seqlen;
+  const size_t row = (size_t)c.head_dim * 2;
+  m.kv_bytes = align_up((size_t)c.heads * m.cap * row);                     // one of K/V, one layer
+  m.raw_bytes = align_up((size_t)c.heads * raw_frames * c.frame_seqlen * row);
+  m.q_bytes = align_up((size_t)c.heads * m.q_stride * row);
+  m.lse_bytes = align_up((size_t)c.heads * m.q_stride * 4);
+  m.score_bytes = align_up((size_t)m.cap * 4);
+  m.tab_t = align_up((size_t)c.t_max * m.pt * 8);
+  m.tab_h = align_up((size_t)c.grid_h * m.ph * 8);
+  m.tab_w = align_up((size_t)c.grid_w * m.pw * 8);
+  m.status_bytes = kAlign;
+  const int nraw = c.policy == RC_ROLLING_SINK ? 2 : (c.policy == RC_INFINITY_ROPE ? 1 : 0);
+  size_t o = 0;
+  m.off_kv = o;
+  o += 2 * m.kv_bytes * c.layers;
+  m.off_raw = o;
+  o += (size_t)nraw * m.raw_bytes * c.layers;
+  m.off_q = o;
+  o += m.q_bytes;
+  m.off_lse = o;
+  o += m.lse_bytes;
+  m.off_score_phys = o;
+  o += m.score_bytes;
+  m.off_score_logical = o;
+  o += m.score_bytes;
+  m.off_tab_t = o;
+  o += m.tab_t;
+  m.off_tab_h = o;
+  o += m.tab_h;
+  m.off_tab_w = o;
+  o += m.tab_w;
+  m.off_status = o;
+  o += m.status_bytes;
+  m.total = o;
+  return m;
+}
+
+// fp64 cos/sin of pos * theta^(-2j / (2 P)) for pos in [0, n_pos), rounded to fp32.
+void build_table(std::vector<float>& out, int n_pos, int pairs, double theta) {
+  out.assign((size_t)n_pos * pairs * 2, 0.f);
+  for (int j = 0; j < pairs; ++j) {
+    const double omega = std::pow(theta, -2.0 * j / (2.0 * pairs));
+    for (int t = 0; t < n_pos; ++t) {
+      const double a = t * omega;
+      out[((size_t)t * pairs + j) * 2] = (float)std::cos(a);
+      out[((size_t)t * pairs + j) * 2 + 1] = (float)std::sin(a);
+    }
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [heads][rows][d] bf16, head stride `head_stride_rows` rows; box {64, 128, 1}, 128B swizzle.
+rc_status make_map(CUtensorMap* map, void* base, int d, int rows, int heads, long long head_stride_rows) {
+  auto fn = encode_fn();
+  if (!fn) return set_err(RC_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)head_stride_rows * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_err(RC_ECUDA, "cuTensorMapEncodeTiled failed: " + std::to_string(r));
+  return RC_OK;
+}
+
+struct Cache {
+  rc_config cfg{};
+  std::unique_ptr<rc::Engine> engine;
+  bool device = false;
+  uint8_t* mem = nullptr;
+  MemPlan mp{};
+  std::vector<uint16_t*> kc, vc, rawk, rawv;
+  std::vector<CUtensorMap> tm_k, tm_v;
+  CUtensorMap tm_q{};
+  int tm_q_rows = -1;
+  std::vector<float> tab[3];
+  rc::RopeTables rt{};
+  uint16_t* qrot = nullptr;
+  float* lse_scratch = nullptr;
+  float* score_phys = nullptr;
+  float* score_logical = nullptr;
+  int* status = nullptr;
+};
+
+rc_status check_handle(const void* h) {
+  if (!h) return set_err(RC_EINVAL, "null handle");
+  return RC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rc_last_error(void) { return g_err.c_str(); }
+
+rc_status rc_config_init(rc_config* cfg, int layers, int heads, int head_dim, int frame_seqlen,
+                         int sink_frames, int window_frames) {
+  if (!cfg) return set_err(RC_EINVAL, "null config");
+  std::memset(cfg, 0, sizeof(*cfg));
+  cfg->layers = layers;
+  cfg->heads = heads;
+  cfg->head_dim = head_dim;
+  cfg->frame_seqlen = frame_seqlen;
+  cfg->grid_h = 1;
+  cfg->grid_w = frame_seqlen;
+  cfg->sink_frames = sink_frames;
+  cfg->window_frames = window_frames;
+  cfg->chunk_frames = 3;
+  cfg->mask_block_frames = 1;
+  cfg->theta = 10000.0;
+  cfg->t_max = 4096;
+  cfg->policy = RC_SLIDING;
+  return RC_OK;
+}
+
+rc_status rc_cache_bytes(const rc_config* cfg, size_t* bytes) {
+  if (!cfg || !bytes) return set_err(RC_EINVAL, "null argument");
+  std::string err;
+  if (rc_status st = rc::ValidateConfig(*cfg, &err)) return set_err(st, err);
+  rc::Engine e(*cfg);
+  *bytes = plan_memory(*cfg, e.pristine_frames()).total;
+  return RC_OK;
+}
+
+rc_status rc_cache_create(const rc_config* cfg, void* dev_mem, size_t bytes, void** out_handle) {
+  if (!cfg || !out_handle) return set_err(RC_EINVAL, "null argument");
+  *out_handle = nullptr;
+  std::string err;
+  if (rc_status st = rc::ValidateConfig(*cfg, &err)) return set_err(st, err);
+  auto c = std::make_unique<Cache>();
+  c->cfg = *cfg;
+  c->engine = std::make_unique<rc::Engine>(*cfg);
+  c->mp = plan_memory(*cfg, c->engine->pristine_frames());
+  const MemPlan& m = c->mp;
+  build_table(c->tab[0], cfg->t_max, m.pt, cfg->theta);
+  build_table(c->tab[1], cfg->grid_h, m.ph, cfg->theta);
+  build_table(c->tab[2], cfg->grid_w, m.pw, cfg->theta);
+  if (dev_mem) {
+    if (bytes < m.total) return set_err(RC_ENOMEM, "memory block smaller than rc_cache_bytes()");
+    if (reinterpret_cast<uintptr_t>(dev_mem) % kAlign) return set_err(RC_EINVAL, "memory block must be 256-byte aligned");
+    c->device = true;
+    c->mem = static_cast<uint8_t*>(dev_mem);
+    uint8_t* b = c->mem;
+    const int L = cfg->layers;
+    const int nraw = cfg->policy == RC_ROLLING_SINK ? 2 : (cfg->policy == RC_INFINITY_ROPE ? 1 : 0);
+    for (int l = 0; l < L; ++l) {
+      c->kc.push_back(reinterpret_cast<uint16_t*>(b + m.off_kv + (2 * (size_t)l) * m.kv_bytes));
+      c->vc.push_back(reinterpret_cast<uint16_t*>(b + m.off_kv + (2 * (size_t)l + 1) * m.kv_bytes));
+      c->rawk.push_back(nraw >= 1 ? reinterpret_cast<uint16_t*>(b + m.off_raw + (nraw * (size_t)l) * m.raw_bytes)
+                                  : nullptr);
+      c->rawv.push_back(nraw == 2 ? reinterpret_cast<uint16_t*>(b + m.off_raw + (nraw * (size_t)l + 1) * m.raw_bytes)
+                                  : nullptr);
+    }
+    c->qrot = reinterpret_cast<uint16_t*>(b + m.off_q);
+    c->lse_scratch = reinterpret_cast<float*>(b + m.off_lse);
+    c->score_phys = reinterpret_cast<float*>(b + m.off_score_phys);
+    c->score_logical = reinterpret_cast<float*>(b + m.off_score_logical);
+    c->status = reinterpret_cast<int*>(b + m.off_status);
+    cudaError_t e = cudaMemset(c->mem, 0, m.total);
+    if (e != cudaSuccess) return cuda_err(e, "cudaMemset");
+    float* tabs[3] = {reinterpret_cast<float*>(b + m.off_tab_t), reinterpret_cast<float*>(b + m.off_tab_h),
+                      reinterpret_cast<float*>(b + m.off_tab_w)};
+    for (int a = 0; a < 3; ++a) {
+      if (c->tab[a].empty()) continue;
+      e = cudaMemcpy(tabs[a], c->tab[a].data(), c->tab[a].size() * 4, cudaMemcpyHostToDevice);
+      if (e != cudaSuccess) return cuda_err(e, "cudaMemcpy tables");
+    }
+    c->rt = rc::RopeTables{reinterpret_cast<const float2*>(tabs[0]), reinterpret_cast<const float2*>(tabs[1]),
+                           reinterpret_cast<const float2*>(tabs[2]), m.pt, m.ph, m.pw, cfg->grid_w, cfg->t_max};
+    c->tm_k.resize(L);
+    c->tm_v.resize(L);
+    for (int l = 0; l < L; ++l) {
+      if (rc_status st = make_map(&c->tm_k[l], c->kc[l], cfg->head_dim, m.cap, cfg->heads, m.cap)) return st;
+      if (rc_status st = make_map(&c->tm_v[l], c->vc[l], cfg->head_dim, m.cap, cfg->heads, m.cap)) return st;
+    }
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_err(e, "cache init");
+  }
+  *out_handle = c.release();
+  return RC_OK;
+}
+
+rc_status rc_cache_destroy(void* handle) {
+  delete static_cast<Cache*>(handle);
+  return RC_OK;
+}
+
+rc_status rc_reindex(void* handle, rc_policy policy, int t_delta, unsigned flags, void* stream) {
+  (void)stream;
+  if (rc_status st = check_handle(handle)) return st;
+  Cache* c = static_cast<Cache*>(handle);
+  if (policy != c->cfg.policy) return set_err(RC_EINVAL, "policy differs from the cache's policy");
+  std::string err;
+  if (rc_status st = c->engine->Reindex(t_delta, flags, &err)) return set_err(st, err);
+  return RC_OK;
+}
+
+rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, const void* v_new, int frame_start,
+                  int n_frames, rc_policy policy, void* out, float* lse, float* scores, int32_t* topc, int C,
+                  void* stream) {
+  if (rc_status st = check_handle(handle)) return st;
+  Cache* c = static_cast<Cache*>(handle);
+  const rc_config& cfg = c->cfg;
+  if (policy != cfg.policy) return set_err(RC_EINVAL, "policy differs from the cache's policy");
+  if (C < 0 || (C > 0 && !topc) || (topc && C == 0)) return set_err(RC_EINVAL, "topc needs C > 0");
+  if (c->device) {
+    if (!q || !k_new || !v_new || !out) return set_err(RC_EINVAL, "null tensor");
+    for (const void* ptr : {q, k_new, v_new, (const void*)out})
+      if (reinterpret_cast<uintptr_t>(ptr) % 16) return set_err(RC_EINVAL, "tensors must be 16-byte aligned");
+  } else if (q || k_new || v_new || out || lse || scores || topc) {
+    return set_err(RC_EINVAL, "a host-only handle takes no tensors");
+  }
+  rc::StepPlan plan;
+  std::string err;
+  if (rc_status st = c->engine->Step(layer, frame_start, n_frames, &plan, &err)) return set_err(st, err);
+  if (!c->device) return RC_OK;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const MemPlan& m = c->mp;
+  const int F = cfg.frame_seqlen, H = cfg.heads, d = cfg.head_dim;
+  const int Nq = n_frames * F;
+
+  // K2: re-rotation jobs (before the append; they touch other slots)
+  for (size_t j0 = 0; j0 < plan.jobs.size(); j0 += rc::kMaxJobs) {
+    rc::RerotateParams rp{};
+    rp.kc = c->kc[layer];
+    rp.vc = c->vc[layer];
+    rp.raw_k = c->rawk[layer];
+    rp.raw_v = c->rawv[layer];
+    rp.H = H;
+    rp.d = d;
+    rp.F = F;
+    rp.cap = m.cap;
+    rp.raw_cap = m.raw_frames * F;
+    rp.n_jobs = (int)std::min<size_t>(rc::kMaxJobs, plan.jobs.size() - j0);
+    for (int j = 0; j < rp.n_jobs; ++j) {
+      const rc::Job& jb = plan.jobs[j0 + j];
+      rp.job[j] = rc::RerotateJob{jb.dst_slot, jb.mode, jb.src_frame, jb.sigma, jb.delta, jb.copy_v};
+    }
+    rp.rt = c->rt;
+    if (cudaError_t e = rc::launch_rerotate(rp, s)) return cuda_err(e, "rerotate launch");
+  }
+
+  // K1: fused RoPE + append
+  rc::AppendParams ap{};
+  ap.q = static_cast<const uint16_t*>(q);
+  ap.k = static_cast<const uint16_t*>(k_new);
+  ap.v = static_cast<const uint16_t*>(v_new);
+  ap.q_rot = c->qrot;
+  ap.kc = c->kc[layer];
+  ap.vc = c->vc[layer];
+  ap.raw_k = c->rawk[layer];
+  ap.raw_v = c->rawv[layer];
+  ap.n_tok = Nq;
+  ap.H = H;
+  ap.d = d;
+  ap.F = F;
+  ap.cap = m.cap;
+  ap.q_stride = m.q_stride;
+  ap.raw_cap = m.raw_frames * F;
+  ap.n_frames = n_frames;
+  for (int r = 0; r < n_frames; ++r) {
+    ap.slot[r] = plan.append[r].slot;
+    ap.sigma[r] = plan.append[r].sigma;
+    ap.raw_frame[r] = plan.append[r].raw_frame;
+  }
+  ap.rt = c->rt;
+  if (cudaError_t e = rc::launch_append(ap, s)) return cuda_err(e, "append launch");
+
+  // K4: attention
+  if (c->tm_q_rows != Nq) {
+    if (rc_status st = make_map(&c->tm_q, c->qrot, d, Nq, H, m.q_stride)) return st;
+    c->tm_q_rows = Nq;
+  }
+  const bool want_scores = scores || topc;
+  float* lse_buf = lse ? lse : (want_scores ? c->lse_scratch : nullptr);
+  rc::AttnParams at;
+  std::memset(&at, 0, sizeof(at));
+  at.tm_q = c->tm_q;
+  at.tm_k = c->tm_k[layer];
+  at.tm_v = c->tm_v[layer];
+  at.out = static_cast<uint16_t*>(out);
+  at.lse = lse_buf;
+  at.status = c->status;
+  at.Nq = Nq;
+  at.H = H;
+  at.F = F;
+  at.mask_block = cfg.mask_block_frames;
+  at.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
+  if (plan.segs.size() > (size_t)rc::kMaxSegs) return set_err(RC_ERANGE, "too many KV segments");
+  at.n_segs = (int)plan.segs.size();
+  for (int i = 0; i < at.n_segs; ++i)
+    at.seg[i] = rc::KvSegment{plan.segs[i].tok_start, plan.segs[i].len, plan.segs[i].rank};
+  if (cudaError_t e = rc::launch_attention(at, d, s)) return cuda_err(e, "attention launch");
+
+  // K6: scores over history tokens + top-C
+  if (want_scores) {
+    std::vector<int> slots;
+    for (auto& cf : plan.cand) slots.push_back(cf.slot);
+    std::sort(slots.begin(), slots.end());
+    rc::ScoreParams sp;
+    std::memset(&sp, 0, sizeof(sp));
+    for (size_t i = 0; i < slots.size();) {
+      size_t j = i + 1;
+      while (j < slots.size() && slots[j] == slots[j - 1] + 1) ++j;
+      if (sp.n_segs == rc::kMaxSegs) return set_err(RC_ERANGE, "too many candidate segments");
+      sp.seg[sp.n_segs++] = rc::KvSegment{slots[i] * F, (int)(j - i) * F, -1};
+      i = j;
+    }
+    if (cudaError_t e = cudaMemsetAsync(c->score_phys, 0, (size_t)m.cap * 4, s)) return cuda_err(e, "memset");
+    sp.tm_q = c->tm_q;
+    sp.tm_k = c->tm_k[layer];
+    sp.lse = lse_buf;
+    sp.score_phys = c->score_phys;
+    sp.status = c->status;
+    sp.Nq = Nq;
+    sp.H = H;
+    sp.scale_log2 = at.scale_log2;
+    if (cudaError_t e = rc::launch_scores(sp, d, s)) return cuda_err(e, "scores launch");
+    rc::TopCParams tp;
+    std::memset(&tp, 0, sizeof(tp));
+    tp.score_phys = c->score_phys;
+    tp.scores_out = scores ? scores : c->score_logical;
+    tp.topc = topc;
+    tp.C = C;
+    tp.F = F;
+    tp.n_cand_frames = (int)plan.cand.size();
+    for (size_t i = 0; i < plan.cand.size(); ++i) {
+      tp.cand_slot[i] = plan.cand[i].slot;
+      tp.cand_lpos[i] = plan.cand[i].lpos;
+    }
+    if (cudaError_t e = rc::launch_topc(tp, s)) return cuda_err(e, "topc launch");
+  }
+  return RC_OK;
+}
+
+rc_status rc_get_state(const void* handle, int layer, rc_state* out) {
+  if (rc_status st = check_handle(handle)) return st;
+  if (!out) return set_err(RC_EINVAL, "null state");
+  const Cache* c = static_cast<const Cache*>(handle);
+  if (layer < 0 || layer >= c->cfg.layers) return set_err(RC_EINVAL, "layer out of range");
+  const rc::LayerState& L = c->engine->layer(layer);
+  std::memset(out, 0, sizeof(*out));
+  out->n_kept = (int)L.kept.size();
+  out->frames_committed = L.end;
+  out->chunk_start = L.cur_start;
+  out->chunk_frames = L.cur_n;
+  out->valid_tokens = (int)L.kept.size() * c->cfg.frame_seqlen;
+  out->shift = L.shift;
+  out->n_jobs = L.n_jobs;
+  int nc = 0;
+  for (size_t e = 0; e < L.kept.size(); ++e) {
+    const rc::Kept& k = L.kept[e];
+    out->kept[e] = rc_frame_state{k.content, k.tau, k.region, k.rank, L.kept_slot[e], k.tau + L.shift};
+    if (k.region == rc::kHist) nc += c->cfg.frame_seqlen;
+  }
+  out->n_candidates = nc;
+  out->n_evicted = (int)L.evicted.size();
+  for (size_t i = 0; i < L.evicted.size() && i < RC_MAX_SLOTS; ++i) out->evicted[i] = L.evicted[i];
+  return RC_OK;
+}
+
+rc_status rc_device_status(void* handle, void* stream) {
+  if (rc_status st = check_handle(handle)) return st;
+  Cache* c = static_cast<Cache*>(handle);
+  if (!c->device) return RC_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaError_t e = cudaStreamSynchronize(s)) return cuda_err(e, "stream sync");
+  int word = 0;
+  if (cudaError_t e = cudaMemcpy(&word, c->status, 4, cudaMemcpyDeviceToHost)) return cuda_err(e, "status read");
+  if (word) {
+    cudaMemset(c->status, 0, 4);
+    return set_err(RC_ETIMEOUT, "a device-side wait gave up (status word " + std::to_string(word) + ")");
+  }
+  return RC_OK;
+}
+
+rc_status rc_cache_layout(const void* handle, rc_layout* out) {
+  if (rc_status st = check_handle(handle)) return st;
+  if (!out) return set_err(RC_EINVAL, "null layout");
+  const Cache* c = static_cast<const Cache*>(handle);
+  const MemPlan& m = c->mp;
+  const int nraw = c->cfg.policy == RC_ROLLING_SINK ? 2 : (c->cfg.policy == RC_INFINITY_ROPE ? 1 : 0);
+  std::memset(out, 0, sizeof(*out));
+  out->kv_layer_stride = 2 * m.kv_bytes;
+  out->k_offset = m.off_kv;
+  out->v_offset = m.off_kv + m.kv_bytes;
+  out->raw_layer_stride = nraw * m.raw_bytes;
+  out->raw_k_offset = nraw >= 1 ? m.off_raw : 0;
+  out->raw_v_offset = nraw == 2 ? m.off_raw + m.raw_bytes : 0;
+  out->q_offset = m.off_q;
+  out->capacity = m.cap;
+  out->raw_frames = m.raw_frames;
+  out->total = m.total;
+  return RC_OK;
+}
+
+rc_status rc_watchdog_selftest(void* handle, unsigned limit_us, void* stream) {
+  if (rc_status st = check_handle(handle)) return st;
+  Cache* c = static_cast<Cache*>(handle);
+  if (!c->device) return set_err(RC_EINVAL, "host-only handle");
+  if (limit_us == 0 || limit_us > 5000000u) return set_err(RC_EINVAL, "limit_us must be in (0, 5e6]");
+  if (cudaError_t e = rc::launch_watchdog_selftest(c->status, limit_us, static_cast<cudaStream_t>(stream)))
+    return cuda_err(e, "watchdog launch");
+  return RC_OK;
+}
+
+rc_status rc_rope_table(const void* handle, int axis, float* dst, size_t* count) {
+  if (rc_status st = check_handle(handle)) return st;
+  if (axis < 0 || axis > 2 || !count) return set_err(RC_EINVAL, "bad axis or count");
+  const Cache* c = static_cast<const Cache*>(handle);
+  const std::vector<float>& t = c->tab[axis];
+  if (!dst) {
+    *count = t.size();
+    return RC_OK;
+  }
+  size_t n = std::min(*count, t.size());
+  std::memcpy(dst, t.data(), n * 4);
+  *count = n;
+  return RC_OK;
+}
+
+}  // extern "C"

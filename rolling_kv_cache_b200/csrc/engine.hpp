@@ -1,0 +1,125 @@
+// Policy engine: the integer side of one rc_step.
+//
+// Host-only C++ (no CUDA). Per layer it keeps the stream history (virtual
+// time of every committed frame, flush points, cut total) and the ring
+// buffer's slot table (which stream frame each physical frame slot holds and
+// the time index its keys are rotated to). A step recomputes the kept frames
+// from the history with the page rules, maps them to slots, and diffs the
+// wanted slot table against the current one to produce the device work:
+// append jobs (fused RoPE + write of the new chunk), re-rotation jobs for
+// kept frames whose time index or content changed, and the attention's KV
+// segment list. Eviction is a slot-table update; no bytes move.
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "../../include/rc.h"
+
+namespace rc {
+
+// Largest number of KV runs one attention launch takes (kernel parameter space).
+constexpr int kEngineMaxSegs = 48;
+
+enum Region { kSink = 0, kHist = 1, kCur = 2 };
+
+struct Kept {
+  int content;  // stream frame index of the raw k/v
+  int tau;      // policy time index
+  int region;   // Region
+  int rank;     // chunk-relative frame for kCur, -1 otherwise
+};
+
+struct Slot {
+  int valid = 0;
+  int content = -1;
+  int sigma = 0;  // time index the stored keys are rotated to
+};
+
+enum JobMode { kRotCopy = 0, kInPlace = 1 };
+
+struct Job {
+  int dst_slot;
+  int mode;       // JobMode
+  int src_frame;  // pristine frame index (kRotCopy)
+  int sigma;      // target time (kRotCopy)
+  int delta;      // time delta (kInPlace)
+  int copy_v;     // kRotCopy also copies V from the pristine source
+};
+
+struct AppendFrame {
+  int slot;
+  int sigma;
+  int raw_frame;  // frame index in the pristine buffer, -1 = none
+};
+
+struct Segment {
+  int tok_start;  // first token (physical, per head) of the run
+  int len;        // tokens
+  int rank;       // mask class of the run: -1 history, else (chunk frame)/mask_block
+};
+
+struct CandFrame {
+  int slot;       // physical slot of a history-region frame
+  int lpos;       // its position in the logical kept list
+};
+
+struct StepPlan {
+  bool repeat = false;
+  int frame_start = 0;
+  int n_frames = 0;
+  AppendFrame append[RC_MAX_CHUNK_FRAMES];
+  std::vector<Job> jobs;
+  std::vector<Segment> segs;
+  std::vector<CandFrame> cand;  // logical order
+};
+
+struct LayerState {
+  int end = 0;
+  int cur_start = -1;
+  int cur_n = 0;
+  std::vector<int> vtime;
+  int cut_total = 0;
+  std::vector<int> flush_points;
+  int sink_delta = 0;
+  int shift = 0;
+  std::vector<Slot> slots;
+  std::vector<Kept> kept;
+  std::vector<int> kept_slot;
+  std::vector<int> evicted;
+  int n_jobs = 0;
+};
+
+class Engine {
+ public:
+  // cfg must already be validated (ValidateConfig).
+  explicit Engine(const rc_config& cfg);
+
+  // Plans and commits one step of `layer`. On failure the layer is unchanged.
+  rc_status Step(int layer, int frame_start, int n_frames, StepPlan* plan, std::string* err);
+  rc_status Reindex(int t_delta, unsigned flags, std::string* err);
+
+  const LayerState& layer(int l) const { return layers_[l]; }
+  int slots() const { return P_; }
+  // Frames of the pristine (raw, unrotated) source a policy keeps: Rolling
+  // Sink's bank of the first K blocks (K and V), Infinity-RoPE's sink (K).
+  int pristine_frames() const;
+  bool pristine_has_v() const { return cfg_.policy == RC_ROLLING_SINK; }
+
+ private:
+  std::vector<Kept> KeptSet(const LayerState& L) const;
+  int SlotOf(const LayerState& L, const Kept& k) const;
+  int ShiftOf(const LayerState& L) const;
+
+  rc_config cfg_;
+  int B_, S_f_, W_f_, P_, F_;
+  std::vector<LayerState> layers_;
+};
+
+// Returns RC_OK or RC_EINVAL with a message.
+rc_status ValidateConfig(const rc_config& cfg, std::string* err);
+// Default RoPE pair split of head_dim/2 pairs.
+void DefaultPairs(int head_dim, int* pt, int* ph, int* pw);
+
+}  // namespace rc

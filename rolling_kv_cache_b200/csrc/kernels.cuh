@@ -1,0 +1,115 @@
+// Kernel parameter blocks and launchers. Every kernel receives its metadata
+// by value (a __grid_constant__ struct), so a step does no host-to-device
+// copy of plans.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/rc.h"
+
+namespace rc {
+
+constexpr int kMaxJobs = 64;
+constexpr int kMaxSegs = 48;  // == kEngineMaxSegs
+constexpr int kMaxCandFrames = RC_MAX_SLOTS;
+
+struct RopeTables {
+  const float2* t;  // [t_max][pt]   (cos, sin)
+  const float2* h;  // [grid_h][ph]
+  const float2* w;  // [grid_w][pw]
+  int pt, ph, pw;
+  int grid_w;
+  int t_max;
+};
+
+// K1: fused RoPE + append of one chunk.
+struct AppendParams {
+  const uint16_t* q;   // [n_tok][H][d]
+  const uint16_t* k;
+  const uint16_t* v;
+  uint16_t* q_rot;     // [H][q_stride][d]
+  uint16_t* kc;        // [H][cap][d]
+  uint16_t* vc;
+  uint16_t* raw_k;     // pristine [H][raw_cap][d] or null
+  uint16_t* raw_v;     // pristine V (Rolling Sink bank) or null
+  int n_tok, H, d, F, cap, q_stride, raw_cap;
+  int n_frames;
+  int slot[RC_MAX_CHUNK_FRAMES];
+  int sigma[RC_MAX_CHUNK_FRAMES];
+  int raw_frame[RC_MAX_CHUNK_FRAMES];
+  RopeTables rt;
+};
+
+// K2: re-rotation jobs (rotate-copy from a pristine source, or in place).
+struct RerotateJob {
+  int dst_slot;
+  int mode;       // 0 rotate-copy, 1 in place (t pairs only)
+  int src_frame;  // pristine frame
+  int sigma;      // target time (rotate-copy)
+  int delta;      // time delta (in place)
+  int copy_v;
+};
+struct RerotateParams {
+  uint16_t* kc;
+  uint16_t* vc;
+  const uint16_t* raw_k;
+  const uint16_t* raw_v;
+  int H, d, F, cap, raw_cap;
+  int n_jobs;
+  RerotateJob job[kMaxJobs];
+  RopeTables rt;
+};
+
+struct KvSegment {
+  int tok_start;
+  int len;
+  int rank;  // -1 history, else mask class of the run
+};
+
+// K4: chunk attention (one CTA per 128-query tile and head).
+struct alignas(64) AttnParams {
+  CUtensorMap tm_q;    // q_rot [H][Nq][d], box {64, 128, 1}, 128B swizzle
+  CUtensorMap tm_k;    // K cache [H][cap][d]
+  CUtensorMap tm_v;    // V cache [H][cap][d]
+  uint16_t* out;       // [Nq][H][d] bf16
+  float* lse;          // [H][Nq] or null
+  int* status;         // device status word
+  int Nq, H, F, mask_block;
+  float scale_log2;    // log2(e) / sqrt(d)
+  int n_segs;
+  KvSegment seg[kMaxSegs];
+};
+
+// K6a: column scores over history tokens (second QK^T pass with final LSE).
+struct alignas(64) ScoreParams {
+  CUtensorMap tm_q;
+  CUtensorMap tm_k;
+  const float* lse;    // [H][Nq] natural log
+  float* score_phys;   // [cap] fp32, accumulated with atomics
+  int* status;
+  int Nq, H;
+  float scale_log2;
+  int n_segs;
+  KvSegment seg[kMaxSegs];
+};
+
+// K6b: gather scores to logical order + top-C.
+struct TopCParams {
+  const float* score_phys;
+  float* scores_out;   // [n_cand] or null
+  int32_t* topc;       // [C] or null
+  int C, F, n_cand_frames;
+  int cand_slot[kMaxCandFrames];
+  int cand_lpos[kMaxCandFrames];
+};
+
+cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+cudaError_t launch_rerotate(const RerotateParams& p, cudaStream_t s);
+cudaError_t launch_attention(const AttnParams& p, int head_dim, cudaStream_t s);
+cudaError_t launch_scores(const ScoreParams& p, int head_dim, cudaStream_t s);
+cudaError_t launch_topc(const TopCParams& p, cudaStream_t s);
+cudaError_t launch_watchdog_selftest(int* status, unsigned limit_us, cudaStream_t s);
+
+}  // namespace rc

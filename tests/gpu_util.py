@@ -1,0 +1,146 @@
+"""Helpers for the GPU tests: device tensors from seeded inputs, a CPU fp32
+restatement of the RoPE kernels' arithmetic (for bit-exact checks), and a
+stream driver that runs a workload through the library and the oracle side
+by side."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import rc_synth
+from oracle import OracleStream
+from rolling_kv_cache_b200 import binding as B
+from rolling_kv_cache_b200.cache import RollingKVCache
+
+from rcutil import config_for, lib_kept, oracle_kept
+
+TOL_MAX, TOL_MEAN, TOL_LSE = 2e-2, 2e-3, 1e-2
+
+
+def dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def bits_of(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def f32(bits):
+    return rc_synth.bf16_bits_to_f32(bits)
+
+
+def rope_fp32(x_bits, t_pos, h_pos, w_pos, tables, pairs):
+    """The kernels' rotation restated in numpy fp32: x [n, H, d] bf16 bits."""
+    pt, ph, pw = pairs
+    x = f32(x_bits).astype(np.float32)
+    n, H, d = x.shape
+    c = np.empty((n, d // 2), np.float32)
+    s = np.empty((n, d // 2), np.float32)
+    tt, th, tw = (tb.reshape(-1, P, 2) for tb, P in zip(tables, pairs))
+    c[:, :pt], s[:, :pt] = tt[t_pos, :, 0], tt[t_pos, :, 1]
+    c[:, pt:pt + ph], s[:, pt:pt + ph] = th[h_pos, :, 0], th[h_pos, :, 1]
+    c[:, pt + ph:], s[:, pt + ph:] = tw[w_pos, :, 0], tw[w_pos, :, 1]
+    c, s = c[:, None, :], s[:, None, :]
+    xe, xo = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = (xe * c).astype(np.float32) - (xo * s).astype(np.float32)
+    out[..., 1::2] = (xe * s).astype(np.float32) + (xo * c).astype(np.float32)
+    return rc_synth.f32_to_bf16_bits(out.astype(np.float32))
+
+
+def rope_fp32_delta(x_bits, delta, tables, pairs):
+    """In-place time re-rotation by delta on the t pairs only (fp32 restatement)."""
+    pt = pairs[0]
+    x = f32(x_bits).astype(np.float32)
+    tt = tables[0].reshape(-1, pt, 2)
+    c = tt[abs(delta), :, 0].astype(np.float32)
+    s = (np.float32(-1.0 if delta < 0 else 1.0) * tt[abs(delta), :, 1]).astype(np.float32)
+    xe, xo = x[..., 0:2 * pt:2].copy(), x[..., 1:2 * pt:2].copy()
+    x[..., 0:2 * pt:2] = (xe * c).astype(np.float32) - (xo * s).astype(np.float32)
+    x[..., 1:2 * pt:2] = (xe * s).astype(np.float32) + (xo * c).astype(np.float32)
+    return rc_synth.f32_to_bf16_bits(x.astype(np.float32))
+
+
+def compare(o_gpu, lse_gpu, ref, rows, heads):
+    """Float parity bar: O max-abs / mean-abs and LSE max-abs against fp64."""
+    og = f32(o_gpu)[rows][:, heads].astype(np.float64)
+    err = np.abs(og - ref["o"])
+    lg = lse_gpu[heads][:, rows]
+    lerr = np.abs(lg - ref["lse"])
+    return err.max(), err.mean(), lerr.max()
+
+
+class Runner:
+    """Runs one layer of a workload through the library and the oracle."""
+
+    def __init__(self, w: rc_synth.Workload, layer: int = 0, seed: int = 0, layers=None):
+        self.w = w
+        self.layer = layer
+        self.seed = seed
+        cfg = config_for(w, layers=layers if layers is not None else w.layers)
+        self.cache = RollingKVCache(cfg)
+        self.oracle = OracleStream(w, layer=layer, seed=seed)
+        self.pairs = (cfg.rope_t_pairs, cfg.rope_h_pairs, cfg.rope_w_pairs)
+        if self.pairs == (0, 0, 0):
+            from oracle import rope_pair_split
+            self.pairs = rope_pair_split(w.head_dim)
+        self.tables = [B.rc_rope_table(self.cache.handle, a) for a in range(3)]
+        self.last = None
+
+    def step(self, chunk: int, pass_: int, cut: bool = False, scores: bool = False):
+        w = self.w
+        if cut:
+            self.cache.reindex(w.cut_delta, B.RC_REINDEX_FLUSH | B.RC_REINDEX_CUT)
+            self.oracle.reindex(1 | 2, w.cut_delta)
+        q, k, v = rc_synth.chunk_qkv(w, self.layer, chunk, pass_, self.seed)
+        Nq = q.shape[0]
+        lse = torch.empty((w.heads, Nq), dtype=torch.float32, device="cuda")
+        sc = tc = None
+        if scores:
+            sc = torch.full((w.footprint_tokens,), -1.0, dtype=torch.float32, device="cuda")
+            tc = torch.full((w.topc,), -7, dtype=torch.int32, device="cuda")
+        out = self.cache.step(self.layer, dev_bf16(q), dev_bf16(k), dev_bf16(v),
+                              chunk * w.chunk_frames, lse=lse, scores=sc, topc=tc, C=w.topc if scores else 0)
+        kept = self.oracle.step(chunk, pass_)
+        torch.cuda.synchronize()
+        self.cache.device_status()
+        st = self.cache.state(self.layer)
+        assert lib_kept(st) == oracle_kept(kept)
+        self.last = dict(q=q, k=k, v=v, out=bits_of(out), lse=lse.cpu().numpy(), state=st,
+                         scores=None if sc is None else sc.cpu().numpy()[:st.n_candidates],
+                         topc=None if tc is None else tc.cpu().numpy())
+        return self.last
+
+    def check_append_bitexact(self):
+        """Current chunk's K/V slots == fp32 restatement of RoPE(k) / raw v."""
+        w, st, last = self.w, self.last["state"], self.last
+        F = w.frame_seqlen
+        kc, vc = self.cache.cache_views(self.layer)
+        n = np.arange(F)
+        hh, ww = n // w.grid_w, n % w.grid_w
+        for e in st.kept[:st.n_kept]:
+            if e.region != 2:
+                continue
+            r = e.rank
+            sl = slice(r * F, (r + 1) * F)
+            want_k = rope_fp32(last["k"][sl], np.full(F, e.stored_time), hh, ww, self.tables, self.pairs)
+            got_k = bits_of(kc[:, e.slot * F:(e.slot + 1) * F]).transpose(1, 0, 2)
+            assert np.array_equal(got_k, want_k), ("K slot", e.slot)
+            got_v = bits_of(vc[:, e.slot * F:(e.slot + 1) * F]).transpose(1, 0, 2)
+            assert np.array_equal(got_v, last["v"][sl]), ("V slot", e.slot)
+        qr = bits_of(self.cache.q_rot_view(w.query_tokens)).transpose(1, 0, 2)
+        cur = {e.rank: e.stored_time for e in st.kept[:st.n_kept] if e.region == 2}
+        tq = np.repeat([cur[r] for r in range(w.chunk_frames)], F)
+        want_q = rope_fp32(last["q"], tq, np.tile(hh, w.chunk_frames), np.tile(ww, w.chunk_frames),
+                           self.tables, self.pairs)
+        assert np.array_equal(qr, want_q)
+
+    def check_float(self, rows=None, heads=None, scores=False):
+        ref = self.oracle.outputs(heads=heads, rows=rows, want_scores=scores)
+        rows = ref["rows"]
+        mx, mean, lmx = compare(self.last["out"], self.last["lse"], ref, rows, ref["heads"])
+        assert mx <= TOL_MAX and mean <= TOL_MEAN and lmx <= TOL_LSE, (mx, mean, lmx)
+        return ref, (mx, mean, lmx)
+
+    def close(self):
+        self.cache.close()

@@ -1,0 +1,26 @@
+"""Test helpers: library config from a workload, state comparisons."""
+import rc_synth
+from rolling_kv_cache_b200 import binding as B
+from rolling_kv_cache_b200.cache import make_config
+
+REGION = {0: "sink", 1: "hist", 2: "cur"}
+
+
+def config_for(w: rc_synth.Workload, **over):
+    kw = dict(layers=w.layers, heads=w.heads, head_dim=w.head_dim, grid_h=w.grid_h,
+              grid_w=w.grid_w, sink_frames=w.sink_frames, window_frames=w.window_frames,
+              chunk_frames=w.chunk_frames, policy=w.policy, mask_block_frames=w.mask_block_frames,
+              theta=w.theta, t_max=w.t_max, rs_bank_blocks=w.rs_bank_blocks,
+              rs_sink_blocks=w.rs_sink_blocks, rs_static_semantics=w.rs_static_semantics,
+              ir_f_limit=w.ir_f_limit, ir_sink_blocks=w.ir_sink_blocks,
+              ir_cache_blocks=w.ir_cache_blocks)
+    kw.update(over)
+    return make_config(**kw)
+
+
+def lib_kept(state):
+    return [(e.content, e.tau, REGION[e.region], e.rank) for e in state.kept[:state.n_kept]]
+
+
+def oracle_kept(kept):
+    return [(k.content, k.tau, k.region, k.rank) for k in kept]

@@ -1,0 +1,88 @@
+"""The C ABI library loads without a GPU and exports what include/rc.h declares."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from rolling_kv_cache_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "rc.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rc_[a-z_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = B.lib()
+    names = declared_functions()
+    assert "rc_step" in names and "rc_cache_create" in names and "rc_reindex" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(B.EXPORTS) <= set(names)
+
+
+def test_struct_sizes_match_header_layout():
+    # rc_config: 21 ints + 1 double, with the double 8-byte aligned
+    assert ctypes.sizeof(B.rc_frame_state) == 24
+    assert ctypes.sizeof(B.rc_state) == 4 * 8 + 4 * 256 + 4 + 24 * 256
+
+
+def test_config_init_and_bytes():
+    cfg = B.rc_config_init(1, 12, 128, 1560, 1, 18)
+    assert (cfg.chunk_frames, cfg.mask_block_frames, cfg.t_max, cfg.policy) == (3, 1, 4096, B.RC_SLIDING)
+    assert cfg.grid_h * cfg.grid_w == 1560
+    n = B.rc_cache_bytes(cfg)
+    kv = 2 * 12 * 19 * 1560 * 128 * 2
+    assert kv <= n < kv + 64 * 2 ** 20
+
+
+@pytest.mark.parametrize("field,value", [("head_dim", 96), ("frame_seqlen", 17), ("chunk_frames", 0),
+                                         ("window_frames", 2), ("t_max", 0), ("heads", 0)])
+def test_invalid_configs_rejected(field, value):
+    cfg = B.rc_config_init(1, 12, 128, 1560, 1, 18)
+    setattr(cfg, field, value)
+    with pytest.raises(B.RcError) as e:
+        B.rc_cache_bytes(cfg)
+    assert e.value.status == B.RC_EINVAL
+    assert B.lib().rc_last_error()
+
+
+def test_host_handle_rejects_tensors_and_policy_mismatch():
+    cfg = B.rc_config_init(1, 2, 64, 16, 1, 6)
+    h = B.rc_cache_create(cfg, 0, 0)
+    try:
+        with pytest.raises(B.RcError):
+            B.rc_step(h, 0, 1234, 0, 0, 0, 3, B.RC_SLIDING, 0)
+        with pytest.raises(B.RcError):
+            B.rc_step(h, 0, 0, 0, 0, 0, 3, B.RC_ROLLING_SINK, 0)
+        B.rc_step(h, 0, 0, 0, 0, 0, 3, B.RC_SLIDING, 0)
+        with pytest.raises(B.RcError) as e:
+            B.rc_step(h, 0, 0, 0, 0, 6, 3, B.RC_SLIDING, 0)
+        assert e.value.status == B.RC_ESTATE
+        with pytest.raises(B.RcError):
+            B.rc_step(h, 1, 0, 0, 0, 3, 3, B.RC_SLIDING, 0)   # layer out of range
+        st = B.rc_get_state(h, 0)
+        assert st.frames_committed == 3 and st.n_kept == 3
+    finally:
+        B.rc_cache_destroy(h)
+
+
+def test_rope_tables_are_fp32_roundings_of_fp64():
+    import numpy as np
+    cfg = B.rc_config_init(1, 2, 128, 1560, 1, 6)
+    cfg.grid_h, cfg.grid_w, cfg.t_max = 30, 52, 400
+    h = B.rc_cache_create(cfg, 0, 0)
+    try:
+        for axis, (n, P) in enumerate(((400, 22), (30, 21), (52, 21))):
+            t = B.rc_rope_table(h, axis).reshape(n, P, 2)
+            pos = np.arange(n)[:, None]
+            om = 10000.0 ** (-np.arange(P) / P)
+            a = pos * om[None, :]
+            assert np.max(np.abs(t[..., 0] - np.cos(a))) < 6e-8
+            assert np.max(np.abs(t[..., 1] - np.sin(a))) < 6e-8
+    finally:
+        B.rc_cache_destroy(h)

@@ -1,0 +1,166 @@
+"""The C++ policy engine (host-only handles) against the fp64 oracle's integer state.
+
+Every step of every workload: kept (content, tau, region, rank) in logical
+order must equal the oracle's bit for bit; the slot table must be a valid
+ring mapping; eviction moves no bytes (slots of persisting frames stay put).
+"""
+import random
+
+import pytest
+
+import rc_synth
+from oracle import PolicyOracle
+from oracle.policy import evicted_contents
+from rolling_kv_cache_b200 import binding as B
+
+from rcutil import config_for, lib_kept, oracle_kept
+
+
+def run_stream(w, steps=None):
+    cfg = config_for(w, layers=1)
+    h = B.rc_cache_create(cfg, 0, 0)
+    pol = PolicyOracle.from_workload(w)
+    P = w.footprint_frames
+    prev_slots = {}
+    prev_kept = []
+    n = 0
+    try:
+        for c, p, g0, cut in rc_synth.stream_schedule(w):
+            if cut:
+                B.rc_reindex(h, w.policy, w.cut_delta, B.RC_REINDEX_FLUSH | B.RC_REINDEX_CUT)
+                pol.reindex(1 | 2, w.cut_delta)
+            B.rc_step(h, 0, 0, 0, 0, g0, w.chunk_frames, w.policy, 0)
+            kept = pol.step(g0, w.chunk_frames)
+            st = B.rc_get_state(h, 0)
+            assert lib_kept(st) == oracle_kept(kept), (c, p)
+            assert st.valid_tokens == len(kept) * w.frame_seqlen
+            slots = [e.slot for e in st.kept[:st.n_kept]]
+            assert len(set(slots)) == len(slots) and all(0 <= s < P for s in slots)
+            for e in st.kept[:st.n_kept]:
+                if e.region == 0:
+                    assert e.slot < w.sink_frames
+                assert e.stored_time == e.tau + st.shift
+            # a frame that stays resident with the same content keeps its slot
+            cur = {(e.content, e.region != 2): e.slot for e in st.kept[:st.n_kept]}
+            for key, s in cur.items():
+                if key in prev_slots and key[1] and w.policy != rc_synth.POLICY_ROLLING_SINK:
+                    assert prev_slots[key] == s
+            if p == 0:
+                assert sorted(st.evicted[:st.n_evicted]) == evicted_contents(prev_kept, kept)
+            prev_slots = {(e.content, True): e.slot for e in st.kept[:st.n_kept]}
+            prev_kept = kept
+            n += 1
+            if steps and n >= steps:
+                break
+    finally:
+        B.rc_cache_destroy(h)
+    return n
+
+
+@pytest.mark.parametrize("name", list(rc_synth.WORKLOADS))
+def test_engine_matches_oracle_every_step(name):
+    w = rc_synth.WORKLOADS[name]
+    assert run_stream(w) == w.chunks * w.passes
+
+
+def test_engine_rolling_sink_static_semantics():
+    w = rc_synth.WORKLOADS["rolling_sink"].replace(rs_static_semantics=1, chunks=40)
+    run_stream(w)
+
+
+def test_engine_block_causal_mask_variant():
+    w = rc_synth.WORKLOADS["tiny"].replace(mask_block_frames=3)
+    run_stream(w)
+
+
+def test_engine_jobs_for_policies():
+    # Infinity-RoPE: sink re-rotated every step once shifting (rotate-copy from
+    # its pristine copy); after a cut the kept last block is re-rotated in place.
+    w = rc_synth.WORKLOADS["infinity_rope"]
+    cfg = config_for(w, layers=1)
+    h = B.rc_cache_create(cfg, 0, 0)
+    jobs = []
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        if cut:
+            B.rc_reindex(h, w.policy, 21, 3)
+        B.rc_step(h, 0, 0, 0, 0, g0, 3, w.policy, 0)
+        jobs.append(B.rc_get_state(h, 0).n_jobs)
+    B.rc_cache_destroy(h)
+    assert jobs[:7] == [0] * 7          # no shift before G'_end > f_limit
+    assert jobs[7] == 3 and jobs[8] == 3 and jobs[26] == 3
+    assert jobs[27] == 6 and jobs[28] == 6 and jobs[32] == 3
+    # Rolling Sink: one bank block copied per step after K
+    w = rc_synth.WORKLOADS["rolling_sink"]
+    h = B.rc_cache_create(config_for(w, layers=1), 0, 0)
+    jobs = []
+    for c in range(30):
+        B.rc_step(h, 0, 0, 0, 0, 3 * c, 3, w.policy, 0)
+        jobs.append(B.rc_get_state(h, 0).n_jobs)
+    B.rc_cache_destroy(h)
+    assert jobs[:7] == [0] * 7 and all(j == 3 for j in jobs[7:])
+
+
+def test_engine_repeat_passes_and_layers_independent():
+    w = rc_synth.WORKLOADS["wan13b"]
+    cfg = config_for(w, layers=3)
+    h = B.rc_cache_create(cfg, 0, 0)
+    try:
+        for c in range(8):
+            for p in range(5):
+                for l in range(3):
+                    B.rc_step(h, l, 0, 0, 0, 3 * c, 3, w.policy, 0)
+                    st = B.rc_get_state(h, l)
+                    if p > 0:
+                        assert st.n_evicted == 0 and st.n_jobs == 0
+        with pytest.raises(B.RcError) as e:
+            B.rc_step(h, 0, 0, 0, 0, 3 * 6, 3, w.policy, 0)   # backwards
+        assert e.value.status == B.RC_ESTATE
+        assert B.rc_get_state(h, 0).chunk_start == 21         # unchanged by the failed call
+    finally:
+        B.rc_cache_destroy(h)
+
+
+def test_engine_sink_reindex_sliding():
+    w = rc_synth.WORKLOADS["tiny"].replace(sink_frames=2)
+    cfg = config_for(w, layers=1)
+    h = B.rc_cache_create(cfg, 0, 0)
+    pol = PolicyOracle.from_workload(w)
+    for c in range(12):
+        if c in (4, 9):
+            B.rc_reindex(h, w.policy, 5 if c == 4 else -2, B.RC_REINDEX_SINK)
+            pol.reindex(4, 5 if c == 4 else -2)
+        B.rc_step(h, 0, 0, 0, 0, 3 * c, 3, w.policy, 0)
+        assert lib_kept(B.rc_get_state(h, 0)) == oracle_kept(pol.step(3 * c, 3))
+    B.rc_cache_destroy(h)
+
+
+def test_engine_fuzz_against_oracle():
+    rng = random.Random(1234)
+    for trial in range(60):
+        B_ = rng.randint(1, 4)
+        pol_kind = rng.choice([0, 1, 2, 3])
+        if pol_kind == 2:
+            K = rng.randint(2, 7)
+            S = rng.randint(1, K - 1)
+            w = rc_synth.WORKLOADS["rolling_sink"].replace(
+                chunk_frames=B_, rs_bank_blocks=K, rs_sink_blocks=S, sink_frames=S * B_,
+                window_frames=(K - S + 1) * B_, chunks=rng.randint(1, 40),
+                rs_static_semantics=rng.randint(0, 1))
+        elif pol_kind == 3:
+            Sb = rng.randint(0, 2)
+            Cb = rng.randint(Sb + 1, Sb + 6)
+            cuts = tuple(sorted(rng.sample(range(1, 40), rng.randint(0, 3))))
+            w = rc_synth.WORKLOADS["infinity_rope"].replace(
+                chunk_frames=B_, ir_sink_blocks=Sb, ir_cache_blocks=Cb, sink_frames=Sb * B_,
+                window_frames=(Cb - Sb + 1) * B_, ir_f_limit=rng.randint(B_, 30),
+                chunks=rng.randint(1, 40), cut_chunks=cuts, cut_delta=rng.randint(0, 25))
+        else:
+            S_f = rng.randint(0, 5)
+            W_f = rng.randint(B_, 20)
+            chunks = rng.randint(1, 30)
+            if pol_kind == 0:
+                W_f = max(W_f, chunks * B_ - S_f + 1)
+            w = rc_synth.WORKLOADS["tiny"].replace(
+                policy=pol_kind, chunk_frames=B_, sink_frames=S_f, window_frames=W_f,
+                chunks=chunks, passes=rng.randint(1, 3), mask_block_frames=rng.randint(1, 3))
+        run_stream(w)

@@ -1,0 +1,217 @@
+"""GPU parity: the library (through its C ABI) against the fp64 oracle.
+
+Integer state is compared bit for bit on every step; K/V appends and
+re-rotations bit for bit against a CPU fp32 restatement of the kernels'
+arithmetic; O / LSE against fp64 within max-abs 2e-2, mean-abs 2e-3 (O) and
+1e-2 (LSE); scores within 1e-3 relative; top-C exactly on the kernel's own
+scores and up to near-ties against fp64.
+"""
+import numpy as np
+import pytest
+import torch
+
+import rc_synth
+from oracle import top_c
+from rolling_kv_cache_b200 import binding as B
+from rolling_kv_cache_b200.cache import RollingKVCache
+
+from gpu_util import Runner, bits_of, dev_bf16, rope_fp32, rope_fp32_delta
+from rcutil import config_for
+
+pytestmark = pytest.mark.gpu
+
+W = rc_synth.WORKLOADS
+
+
+def test_watchdog_reports_timeout_and_context_survives():
+    w = W["tiny"]
+    cache = RollingKVCache(config_for(w))
+    cache.watchdog_selftest(20000)
+    with pytest.raises(B.RcError) as e:
+        cache.device_status()
+    assert e.value.status == B.RC_ETIMEOUT
+    q, k, v = (dev_bf16(x) for x in rc_synth.chunk_qkv(w, 0, 0, 0))
+    out = cache.step(0, q, k, v, 0)
+    torch.cuda.synchronize()
+    cache.device_status()           # cleared, and the context still works
+    assert torch.isfinite(out.float()).all()
+    cache.close()
+
+
+@pytest.mark.parametrize("mask_block", [1, 3])
+def test_tiny_every_step(mask_block):
+    w = W["tiny"].replace(mask_block_frames=mask_block)
+    r = Runner(w)
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        r.step(c, p, cut)
+        r.check_append_bitexact()
+        r.check_float()
+    r.close()
+
+
+def test_unbounded_policy_equals_full_history():
+    w = W["tiny"].replace(policy=rc_synth.POLICY_NONE, window_frames=40, chunks=8)
+    r = Runner(w)
+    for c in range(w.chunks):
+        r.step(c, 0)
+        r.check_float()
+    r.close()
+
+
+@pytest.mark.parametrize("mask_block", [1, 3])
+def test_multi_tile_ragged(mask_block):
+    # F = 200 tokens: a frame is 1.56 tiles, Nq = 600 = 4 tiles + 88 rows,
+    # cache runs end mid-tile; 3 heads of 128.
+    w = rc_synth.Workload(name="ragged", workload_id=11, layers=1, heads=3, head_dim=128, grid_h=10,
+                          grid_w=20, chunk_frames=3, sink_frames=1, window_frames=6,
+                          policy=rc_synth.POLICY_SLIDING, chunks=6, dist="normal_frame_mean",
+                          mask_block_frames=mask_block)
+    r = Runner(w)
+    for c in range(w.chunks):
+        r.step(c, 0)
+        r.check_append_bitexact()
+        r.check_float()
+    r.close()
+
+
+def test_repeat_passes_overwrite():
+    w = rc_synth.Workload(name="passes", workload_id=12, layers=2, heads=2, head_dim=128, grid_h=8,
+                          grid_w=16, chunk_frames=3, sink_frames=1, window_frames=9,
+                          policy=rc_synth.POLICY_SLIDING, chunks=6, passes=3, dist="normal_frame_mean")
+    r = Runner(w, layer=1)
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        r.step(c, p)
+        r.check_float()
+    r.close()
+
+
+def test_rolling_sink_small():
+    w = W["rolling_sink"].replace(heads=2, grid_h=8, grid_w=8, chunks=16)
+    r = Runner(w)
+    for c in range(w.chunks):
+        r.step(c, 0)
+        r.check_append_bitexact()
+        r.check_float()
+        st = r.last["state"]
+        if c >= 7:   # the entering sink block was rotate-copied from the bank
+            kc, vc = r.cache.cache_views(0)
+            rk, rv = r.cache.raw_views(0)
+            F = w.frame_seqlen
+            n = np.arange(F)
+            for e in st.kept[:st.n_kept]:
+                if e.region != 0:
+                    continue
+                got = bits_of(kc[:, e.slot * F:(e.slot + 1) * F]).transpose(1, 0, 2)
+                raw = bits_of(rk[:, e.content * F:(e.content + 1) * F]).transpose(1, 0, 2)
+                want = rope_fp32(raw, np.full(F, e.stored_time), n // w.grid_w, n % w.grid_w,
+                                 r.tables, r.pairs)
+                assert np.array_equal(got, want)
+                gv = bits_of(vc[:, e.slot * F:(e.slot + 1) * F])
+                assert np.array_equal(gv, bits_of(rv[:, e.content * F:(e.content + 1) * F]))
+    r.close()
+
+
+def _topc_checks(w, r, ref):
+    sg = r.last["scores"]
+    sr = ref["scores"]
+    rel = np.abs(sg - sr) / np.maximum(np.abs(sr), 1e-30)
+    assert np.max(np.abs(sg - sr)) <= 1e-3 * max(1.0, np.max(np.abs(sr))), np.max(rel)
+    cand = ref["cand_index"]
+    # (i) selection on the kernel's own fp32 scores is exact
+    want = top_c(sg.astype(np.float32), cand, w.topc)
+    got = r.last["topc"]
+    n = min(w.topc, len(cand))
+    assert np.array_equal(got[:n], want)
+    assert np.all(got[n:] == -1)
+    # (ii) against the fp64 selection, swaps only among near-ties of the C-th score
+    ref_sel = set(ref["topc"].tolist())
+    diff = ref_sel.symmetric_difference(set(want.tolist()))
+    if diff and n < len(cand):
+        kth = np.sort(sr)[::-1][n - 1]
+        pos = {int(c): i for i, c in enumerate(cand)}
+        for c in diff:
+            assert abs(sr[pos[c]] - kth) <= 1e-3 * max(1.0, kth)
+
+
+def test_infinity_rope_small_with_scores():
+    w = W["infinity_rope"].replace(heads=2, grid_h=8, grid_w=8, chunks=18, cut_chunks=(9, 13), topc=100)
+    r = Runner(w)
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        r.step(c, p, cut, scores=True)
+        r.check_append_bitexact()
+        ref, _ = r.check_float(scores=True)
+        _topc_checks(w, r, ref)
+        st = r.last["state"]
+        if c in (9, 10):   # the kept last block before the cut, clamped to time 0
+            assert any(e.region == 1 and e.tau == 0 for e in st.kept[:st.n_kept])
+    r.close()
+
+
+def test_inplace_rerotation_bitexact():
+    # Sliding with a sink time shift: the sink is re-rotated in place by delta.
+    w = W["tiny"].replace(heads=2, head_dim=128, grid_h=4, grid_w=8, sink_frames=2, chunks=6)
+    r = Runner(w)
+    for c in range(4):
+        r.step(c, 0)
+    kc, _ = r.cache.cache_views(0)
+    F = w.frame_seqlen
+    before = bits_of(kc[:, 0:2 * F]).copy()
+    r.cache.reindex(5, B.RC_REINDEX_SINK)
+    r.oracle.reindex(4, 5)
+    r.step(4, 0)
+    after = bits_of(kc[:, 0:2 * F])
+    want = rope_fp32_delta(before.transpose(1, 0, 2), 5, r.tables, r.pairs).transpose(1, 0, 2)
+    assert np.array_equal(after, want)
+    r.check_float()
+    r.step(5, 0)
+    r.check_float()
+    r.close()
+
+
+# ----------------------------------------------------------- full sizes
+SAMPLE_ROWS = np.array([0, 1, 127, 128, 1559, 1560, 1561, 3119, 3120, 4607, 4608, 4679])
+
+
+def _sampled(w, steps, layer=0, layers=None, scores_at=()):
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([SAMPLE_ROWS, rng.integers(0, w.query_tokens, 20)]))
+    r = Runner(w, layer=layer, layers=layers)
+    last_chunk = max(steps)
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        if c > last_chunk:
+            break
+        want_scores = c in scores_at
+        r.step(c, p, cut, scores=want_scores)
+        if c in steps:
+            if p == 0:
+                r.check_append_bitexact()
+            r.check_float(rows=rows)
+            st = r.last["state"]
+            assert st.valid_tokens == min(g0 + 3, w.footprint_frames) * w.frame_seqlen or \
+                w.policy == rc_synth.POLICY_INFINITY_ROPE
+        if want_scores:
+            sg = r.last["scores"]
+            want = top_c(sg, np.arange(len(sg)) + 0, w.topc)  # positions; remapped below
+            cand_lpos = np.nonzero(np.repeat([e.region == 1 for e in r.last["state"].kept[:r.last["state"].n_kept]],
+                                             w.frame_seqlen))[0]
+            assert np.array_equal(r.last["topc"], np.sort(cand_lpos[want]))
+            assert np.all(sg > 0) and sg.sum() < w.heads * w.query_tokens
+    r.close()
+
+
+def test_full_wan13b_sampled():
+    w = W["wan13b"]
+    _sampled(w, steps={0, 1, 5, 6, 7}, layer=29, layers=30)
+
+
+def test_full_large_sampled():
+    _sampled(W["large"], steps={0, 1, 5, 6, 7})
+
+
+def test_full_rolling_sink_sampled():
+    _sampled(W["rolling_sink"], steps={0, 5, 6, 7, 8, 12})
+
+
+def test_full_infinity_rope_sampled():
+    w = W["infinity_rope"].replace(cut_chunks=(9, 27, 60))
+    _sampled(w, steps={0, 6, 7, 9, 10}, scores_at={7, 9, 10})
