@@ -1,0 +1,387 @@
+#!/usr/bin/env python
+"""Benchmark of the chunked attention step over the bounded KV cache.
+
+Workload (default): the Wan2.1-1.3B-shaped sliding-window stream -- 30 layers,
+12 heads x 128, 1560-token frames (30x52 latent grid), 3-frame chunks (4680
+queries), sink 1 frame + window 18 frames (29640 cached tokens per head), 4
+denoise passes + 1 clean cache-refresh pass per chunk. One bench step = one
+chunk through all 30 layers x 5 passes = 150 rc_step calls (each: fused RoPE +
+append, tcgen05 attention). Synthetic seeded inputs (N(0,1) + per-frame mean
+N(0, 0.5), bf16); the cache is driven to steady state (full window) before
+warm-up.
+
+Prints one JSON line. ``value`` is chunk-attention TFLOP/s (algorithmic FLOPs
+4*d*H*visible pairs over the timed region's device time, summed over ranks);
+``frames_per_s_per_layer`` the streamed latent frame rate per layer.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload (one head of one layer-pass per step) on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import rc_synth  # noqa: E402
+
+METRIC = "chunk-attention TFLOP/s vs bf16 peak; streamed latent frames/s per layer"
+UNIT = "TFLOP/s"
+
+
+def visible_pairs(w, n_hist_frames: int) -> int:
+    """(query, key) pairs the chunk attention computes (frame-causal in chunk)."""
+    F, B, m = w.frame_seqlen, w.chunk_frames, w.mask_block_frames
+    pairs = 0
+    for r in range(B):
+        vis = sum(1 for r2 in range(B) if r2 // m <= r // m)
+        pairs += F * (n_hist_frames * F + vis * F)
+    return pairs
+
+
+def attention_flops(w, n_hist_frames: int, heads=None) -> float:
+    return 4.0 * w.head_dim * (w.heads if heads is None else heads) * visible_pairs(w, n_hist_frames)
+
+
+def steady_hist_frames(w) -> int:
+    return w.footprint_frames - w.chunk_frames
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("attn_kernel.cu", "ptx.cuh", "kernels.cuh"):
+        with open(os.path.join(ROOT, "rolling_kv_cache_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def attention_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if it
+    was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "attention_wan13b_ncu.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    sha = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    val = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not sha or not val or sha.group(1) != kernel_source_hash():
+        return None
+    return float(val.group(1))
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", self.gpu_id],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.rows = []
+        if self.proc is None:
+            return False
+        time.sleep(0.3)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+        return False
+
+    def summary(self):
+        if not getattr(self, "rows", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in self.rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        loaded = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+def make_cfg(w, layers=None):
+    from rolling_kv_cache_b200.cache import make_config
+    return make_config(layers=w.layers if layers is None else layers, heads=w.heads,
+                       head_dim=w.head_dim, grid_h=w.grid_h, grid_w=w.grid_w,
+                       sink_frames=w.sink_frames, window_frames=w.window_frames,
+                       chunk_frames=w.chunk_frames, policy=w.policy,
+                       mask_block_frames=w.mask_block_frames, theta=w.theta, t_max=w.t_max,
+                       rs_bank_blocks=w.rs_bank_blocks, rs_sink_blocks=w.rs_sink_blocks,
+                       rs_static_semantics=w.rs_static_semantics, ir_f_limit=w.ir_f_limit,
+                       ir_sink_blocks=w.ir_sink_blocks, ir_cache_blocks=w.ir_cache_blocks)
+
+
+# ------------------------------------------------------------ CPU oracle
+def oracle_sample_seconds(w, heads: int, chunk: int = 7):
+    """Time the fp64 oracle on one layer-pass of a steady-state chunk,
+    restricted to ``heads`` heads. Returns (seconds, flops, threads)."""
+    from oracle import OracleStream
+    st = OracleStream(w, layer=0, seed=0)
+    for c in range(chunk + 1):
+        st.step(c, w.passes - 1 if c < chunk else 0)
+    st.outputs(heads=[0], rows=np.arange(1))       # warm the regenerated inputs
+    t0 = time.perf_counter()
+    st.outputs(heads=list(range(heads)))
+    dt = time.perf_counter() - t0
+    n_hist = sum(1 for k in st.kept if k.region != "cur")
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    return dt, attention_flops(w, n_hist, heads=heads), threads
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    heads = 1
+    for _ in range(args.warmup):
+        oracle_sample_seconds(w, heads)
+    secs, flops = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl, threads = oracle_sample_seconds(w, heads)
+        secs += dt
+        flops += fl
+    value = flops / secs / 1e12
+    sample = (f"fp64 numpy oracle, one head of one layer-pass per step (chunk 7 of {w.name}, "
+              f"{w.query_tokens} queries x {steady_hist_frames(w) * w.frame_seqlen}+ keys)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name}, "cpu_baseline": {
+                "value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------ GPU path
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+    from rolling_kv_cache_b200 import binding as B
+    from rolling_kv_cache_b200.cache import RollingKVCache
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    cache = RollingKVCache(make_cfg(w), dev)
+    stream = torch.cuda.current_stream(dev)
+    # a small pool of distinct seeded inputs, resident in HBM, cycled over
+    # (layer, pass, chunk); timing does not depend on the values
+    pool = []
+    for i in range(6):
+        q, k, v = rc_synth.chunk_qkv(w, i % w.layers, i, i % w.passes, seed=rank)
+        pool.append(tuple(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in (q, k, v)))
+    out = torch.empty_like(pool[0][0])
+    B_ = w.chunk_frames
+    calls_per_step = w.layers * w.passes
+
+    def run_chunk(c):
+        for p in range(w.passes):
+            for l in range(w.layers):
+                q, k, v = pool[(c * 7 + p * 3 + l) % len(pool)]
+                cache.step(l, q, k, v, c * B_, out=out)
+
+    chunk = 0
+    prefill = (w.footprint_frames + B_ - 1) // B_   # until the window is full
+    for _ in range(prefill):
+        run_chunk(chunk)
+        chunk += 1
+    for _ in range(args.warmup):
+        run_chunk(chunk)
+        chunk += 1
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    B.rc_profile_begin(cache.handle, args.steps * calls_per_step * 2 + 16)
+    gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    if not gpu_uuid.startswith("GPU-"):
+        gpu_uuid = "GPU-" + gpu_uuid
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_uuid) as clocks:
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            run_chunk(chunk)
+            chunk += 1
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    prof = B.rc_profile_end(cache.handle)
+    cache.device_status()
+
+    att = prof["attention"]
+    flops_rank = att["flops"]
+    ms_max = ms
+    flops_total = flops_rank
+    if world > 1:
+        t = torch.tensor([ms, flops_rank], dtype=torch.float64, device=dev)
+        mx = t.clone()
+        dist.all_reduce(mx[:1], op=dist.ReduceOp.MAX)
+        dist.all_reduce(t[1:], op=dist.ReduceOp.SUM)
+        ms_max, flops_total = float(mx[0]), float(t[1])
+    value = flops_total / (ms_max / 1e3) / 1e12
+    frames = args.steps * B_ * world
+    frames_per_s_per_layer = frames / (ms_max / 1e3) * w.layers / world
+    launches = sum(v["launches"] for v in prof.values())
+
+    # ---------------- end to end through the public API with host buffers
+    e2e_steps = max(1, args.e2e_steps)
+    host_pool = [tuple(t.cpu().pin_memory() for t in trip) for trip in pool[:3]]
+    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * 2 for t in host_pool[0]) * calls_per_step
+    d2h = out_host.numel() * 2 * calls_per_step
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    e2e_flops = 0.0
+    for _ in range(e2e_steps):
+        for p in range(w.passes):
+            for l in range(w.layers):
+                q, k, v = host_pool[(p + l) % len(host_pool)]
+                cache.step(l, q, k, v, chunk * B_, out=out_host)
+        e2e_flops += attention_flops(w, steady_hist_frames(w)) * calls_per_step
+        chunk += 1
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    e2e_tot = e2e_flops
+    if world > 1:
+        t = torch.tensor([e2e_ms, e2e_flops], dtype=torch.float64, device=dev)
+        mx = t.clone()
+        dist.all_reduce(mx[:1], op=dist.ReduceOp.MAX)
+        dist.all_reduce(t[1:], op=dist.ReduceOp.SUM)
+        e2e_ms, e2e_tot = float(mx[0]), float(t[1])
+    e2e_value = e2e_tot / (e2e_ms / 1e3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    att_ms = att["ms"] / max(1, att["timed"])
+    att_flops_launch = att["flops"] / max(1, att["launches"])
+    achieved = att_flops_launch / (att_ms / 1e3) / 1e12
+    traffic = attention_traffic()
+    app = prof["append"]
+    app_gbs = (app["bytes"] / max(1, app["launches"])) / (app["ms"] / max(1, app["timed"]) / 1e3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, fl, threads = oracle_sample_seconds(w, heads=3)
+        cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"fp64 numpy oracle, 3 of {w.heads} heads of one layer-pass at a "
+                         f"steady-state chunk ({w.query_tokens} queries x "
+                         f"{steady_hist_frames(w) * w.frame_seqlen}+ keys), {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "layers": w.layers, "heads": w.heads,
+                       "head_dim": w.head_dim, "frame_seqlen": w.frame_seqlen,
+                       "chunk_frames": B_, "sink_frames": w.sink_frames,
+                       "window_frames": w.window_frames, "passes_per_chunk": w.passes,
+                       "cached_tokens_per_head": w.footprint_tokens,
+                       "step": f"one chunk x {w.layers} layers x {w.passes} passes",
+                       "parallelism": f"independent stream per GPU x{world}",
+                       "l2": "inputs larger than L2 (182 MB K/V ring per layer, 30 layers cycled)"},
+            "frames_per_s_per_layer": frames_per_s_per_layer,
+            "frames_per_s_model": frames / (ms_max / 1e3),
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                    "path": "RollingKVCache.step with pinned host q/k/v/out"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "attention (tcgen05)",
+                         "peak_source": f"{peak_src} bf16_tflops_sustained",
+                         "frac_of_burst": achieved / float(peaks.get("bf16_tflops", peak)),
+                         "flops_per_launch": att_flops_launch, "ms_per_launch": att_ms},
+            "kernels": {k: {"launches": v["launches"], "ms_per_launch": v["ms"] / max(1, v["timed"])}
+                        for k, v in prof.items() if v["launches"]},
+            "append_gbs": app_gbs, "append_hbm_frac": app_gbs / float(peaks.get("hbm_gbs", 6650.0)),
+            "gpu_launches": launches,
+            "clocks": clocks.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    cache.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="wan13b", choices=list(rc_synth.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the workload's layer count (small profiling runs)")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    w = rc_synth.WORKLOADS[args.workload]
+    if args.layers:
+        w = w.replace(layers=args.layers)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -220,6 +220,25 @@ rc_status rc_cache_layout(const void* handle, rc_layout* out);
  * usable. Faults nothing. */
 rc_status rc_watchdog_selftest(void* handle, unsigned limit_us, void* stream);
 
+/* Per-kernel timing with CUDA events recorded on the launching stream
+ * around every kernel a step enqueues (re-rotation, append, attention,
+ * scores, top-C). rc_profile_begin arms it for up to max_launches launches
+ * (events are created here, not in rc_step); rc_profile_end synchronizes
+ * the recorded events and reports, per kernel kind, the launch count and
+ * the summed device milliseconds, then disarms. Launches beyond the limit
+ * are counted but not timed. */
+enum { RC_KERNEL_REROTATE = 0, RC_KERNEL_APPEND = 1, RC_KERNEL_ATTENTION = 2,
+       RC_KERNEL_SCORES = 3, RC_KERNEL_TOPC = 4, RC_KERNEL_KINDS = 5 };
+typedef struct rc_profile {
+  int64_t launches[RC_KERNEL_KINDS];
+  int64_t timed[RC_KERNEL_KINDS];
+  double ms[RC_KERNEL_KINDS];
+  double flops[RC_KERNEL_KINDS];  /* algorithmic FLOPs (attention: 4*d*H*visible pairs) */
+  double bytes[RC_KERNEL_KINDS];  /* algorithmic HBM bytes (append, re-rotate) */
+} rc_profile;
+rc_status rc_profile_begin(void* handle, int max_launches);
+rc_status rc_profile_end(void* handle, rc_profile* out);
+
 rc_status rc_cache_destroy(void* handle);
 
 /* Message for the calling thread's last failed call ("" if none). */

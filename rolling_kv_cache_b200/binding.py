@@ -65,9 +65,19 @@ class rc_layout(ctypes.Structure):
                 ("raw_frames", ctypes.c_int32), ("total", ctypes.c_size_t)]
 
 
+RC_KERNEL_NAMES = ["rerotate", "append", "attention", "scores", "topc"]
+
+
+class rc_profile(ctypes.Structure):
+    _fields_ = [("launches", ctypes.c_int64 * 5), ("timed", ctypes.c_int64 * 5),
+                ("ms", ctypes.c_double * 5), ("flops", ctypes.c_double * 5),
+                ("bytes", ctypes.c_double * 5)]
+
+
 EXPORTS = ["rc_config_init", "rc_cache_bytes", "rc_cache_create", "rc_step", "rc_reindex",
            "rc_get_state", "rc_device_status", "rc_rope_table", "rc_cache_layout",
-           "rc_watchdog_selftest", "rc_cache_destroy", "rc_last_error"]
+           "rc_watchdog_selftest", "rc_profile_begin", "rc_profile_end", "rc_cache_destroy",
+           "rc_last_error"]
 
 _lib = None
 
@@ -90,6 +100,8 @@ def lib() -> ctypes.CDLL:
         L.rc_rope_table.argtypes = [vp, i, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(sz)]
         L.rc_cache_layout.argtypes = [vp, ctypes.POINTER(rc_layout)]
         L.rc_watchdog_selftest.argtypes = [vp, ctypes.c_uint, vp]
+        L.rc_profile_begin.argtypes = [vp, i]
+        L.rc_profile_end.argtypes = [vp, ctypes.POINTER(rc_profile)]
         L.rc_cache_destroy.argtypes = [vp]
         L.rc_last_error.argtypes = []
         L.rc_last_error.restype = ctypes.c_char_p
@@ -162,6 +174,17 @@ def rc_cache_layout(handle) -> rc_layout:
 
 def rc_watchdog_selftest(handle, limit_us, stream=0) -> None:
     check(lib().rc_watchdog_selftest(handle, limit_us, stream or None))
+
+
+def rc_profile_begin(handle, max_launches) -> None:
+    check(lib().rc_profile_begin(handle, max_launches))
+
+
+def rc_profile_end(handle) -> dict:
+    p = rc_profile()
+    check(lib().rc_profile_end(handle, ctypes.byref(p)))
+    return {n: dict(launches=p.launches[i], timed=p.timed[i], ms=p.ms[i], flops=p.flops[i],
+                    bytes=p.bytes[i]) for i, n in enumerate(RC_KERNEL_NAMES)}
 
 
 def rc_cache_destroy(handle) -> None:

@@ -123,7 +123,47 @@ rc_status make_map(CUtensorMap* map, void* base, int d, int rows, int heads, lon
   return RC_OK;
 }
 
+// Optional per-kernel event timing (rc_profile_begin / rc_profile_end).
+struct Profiler {
+  bool on = false;
+  int max = 0, used = 0;
+  std::vector<cudaEvent_t> ev;  // 2 per timed launch
+  std::vector<int> kind;
+  int64_t launches[RC_KERNEL_KINDS] = {};
+  double flops[RC_KERNEL_KINDS] = {}, bytes[RC_KERNEL_KINDS] = {};
+  void release() {
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);
+    ev.clear();
+    kind.clear();
+    on = false;
+    max = used = 0;
+  }
+  ~Profiler() { release(); }
+};
+
+// Brackets one launch with events when profiling is armed.
+struct Timed {
+  Profiler& p;
+  int k, slot = -1;
+  cudaStream_t s;
+  Timed(Profiler& pr, int kind, cudaStream_t st, double flops, double bytes) : p(pr), k(kind), s(st) {
+    if (!p.on) return;
+    p.launches[k]++;
+    p.flops[k] += flops;
+    p.bytes[k] += bytes;
+    if (p.used < p.max) {
+      slot = p.used++;
+      p.kind[slot] = k;
+      cudaEventRecord(p.ev[2 * slot], s);
+    }
+  }
+  ~Timed() {
+    if (slot >= 0) cudaEventRecord(p.ev[2 * slot + 1], s);
+  }
+};
+
 struct Cache {
+  Profiler prof;
   rc_config cfg{};
   std::unique_ptr<rc::Engine> engine;
   bool device = false;
@@ -298,6 +338,13 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
       rp.job[j] = rc::RerotateJob{jb.dst_slot, jb.mode, jb.src_frame, jb.sigma, jb.delta, jb.copy_v};
     }
     rp.rt = c->rt;
+    double bytes = 0;
+    for (int j = 0; j < rp.n_jobs; ++j) {
+      const rc::RerotateJob& jb = rp.job[j];
+      const double rows = (double)F * H;
+      bytes += jb.mode == 1 ? rows * 2 * (2 * m.pt) * 2 : rows * 2 * d * 2 * (jb.copy_v ? 2 : 1);
+    }
+    Timed tm(c->prof, RC_KERNEL_REROTATE, s, 0.0, bytes);
     if (cudaError_t e = rc::launch_rerotate(rp, s)) return cuda_err(e, "rerotate launch");
   }
 
@@ -325,7 +372,13 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
     ap.raw_frame[r] = plan.append[r].raw_frame;
   }
   ap.rt = c->rt;
-  if (cudaError_t e = rc::launch_append(ap, s)) return cuda_err(e, "append launch");
+  {
+    double bytes = 6.0 * Nq * H * d * 2;
+    for (int r = 0; r < n_frames; ++r)
+      if (ap.raw_frame[r] >= 0) bytes += (double)F * H * d * 2 * (ap.raw_v ? 2 : 1);
+    Timed tm(c->prof, RC_KERNEL_APPEND, s, 0.0, bytes);
+    if (cudaError_t e = rc::launch_append(ap, s)) return cuda_err(e, "append launch");
+  }
 
   // K4: attention
   if (c->tm_q_rows != Nq) {
@@ -351,7 +404,20 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
   at.n_segs = (int)plan.segs.size();
   for (int i = 0; i < at.n_segs; ++i)
     at.seg[i] = rc::KvSegment{plan.segs[i].tok_start, plan.segs[i].len, plan.segs[i].rank};
-  if (cudaError_t e = rc::launch_attention(at, d, s)) return cuda_err(e, "attention launch");
+  {
+    // algorithmic FLOPs: 4 d H per visible (query, key) pair
+    const rc::LayerState& Ls = c->engine->layer(layer);
+    double n_hist = 0;
+    for (const rc::Kept& k : Ls.kept) n_hist += k.region != rc::kCur ? F : 0;
+    double pairs = 0;
+    for (int r = 0; r < n_frames; ++r) {
+      int vis = 0;
+      for (int r2 = 0; r2 < n_frames; ++r2) vis += (r2 / cfg.mask_block_frames) <= (r / cfg.mask_block_frames);
+      pairs += (double)F * (n_hist + (double)vis * F);
+    }
+    Timed tm(c->prof, RC_KERNEL_ATTENTION, s, 4.0 * d * H * pairs, 0.0);
+    if (cudaError_t e = rc::launch_attention(at, d, s)) return cuda_err(e, "attention launch");
+  }
 
   // K6: scores over history tokens + top-C
   if (want_scores) {
@@ -376,7 +442,10 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
     sp.Nq = Nq;
     sp.H = H;
     sp.scale_log2 = at.scale_log2;
-    if (cudaError_t e = rc::launch_scores(sp, d, s)) return cuda_err(e, "scores launch");
+    {
+      Timed tm(c->prof, RC_KERNEL_SCORES, s, 2.0 * d * H * Nq * (double)plan.cand.size() * F, 0.0);
+      if (cudaError_t e = rc::launch_scores(sp, d, s)) return cuda_err(e, "scores launch");
+    }
     rc::TopCParams tp;
     std::memset(&tp, 0, sizeof(tp));
     tp.score_phys = c->score_phys;
@@ -389,7 +458,10 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
       tp.cand_slot[i] = plan.cand[i].slot;
       tp.cand_lpos[i] = plan.cand[i].lpos;
     }
-    if (cudaError_t e = rc::launch_topc(tp, s)) return cuda_err(e, "topc launch");
+    {
+      Timed tm(c->prof, RC_KERNEL_TOPC, s, 0.0, (double)plan.cand.size() * F * 4 * 2);
+      if (cudaError_t e = rc::launch_topc(tp, s)) return cuda_err(e, "topc launch");
+    }
   }
   return RC_OK;
 }
@@ -462,6 +534,54 @@ rc_status rc_watchdog_selftest(void* handle, unsigned limit_us, void* stream) {
   if (limit_us == 0 || limit_us > 5000000u) return set_err(RC_EINVAL, "limit_us must be in (0, 5e6]");
   if (cudaError_t e = rc::launch_watchdog_selftest(c->status, limit_us, static_cast<cudaStream_t>(stream)))
     return cuda_err(e, "watchdog launch");
+  return RC_OK;
+}
+
+rc_status rc_profile_begin(void* handle, int max_launches) {
+  if (rc_status st = check_handle(handle)) return st;
+  Cache* c = static_cast<Cache*>(handle);
+  if (!c->device) return set_err(RC_EINVAL, "host-only handle");
+  if (max_launches < 0 || max_launches > (1 << 20)) return set_err(RC_EINVAL, "max_launches out of range");
+  Profiler& p = c->prof;
+  p.release();
+  p.ev.resize(2 * (size_t)max_launches);
+  for (auto& e : p.ev)
+    if (cudaError_t err = cudaEventCreate(&e)) {
+      p.ev.clear();
+      return cuda_err(err, "cudaEventCreate");
+    }
+  p.kind.assign(max_launches, 0);
+  p.max = max_launches;
+  p.used = 0;
+  std::fill(p.launches, p.launches + RC_KERNEL_KINDS, 0);
+  std::fill(p.flops, p.flops + RC_KERNEL_KINDS, 0.0);
+  std::fill(p.bytes, p.bytes + RC_KERNEL_KINDS, 0.0);
+  p.on = true;
+  return RC_OK;
+}
+
+rc_status rc_profile_end(void* handle, rc_profile* out) {
+  if (rc_status st = check_handle(handle)) return st;
+  if (!out) return set_err(RC_EINVAL, "null profile");
+  Cache* c = static_cast<Cache*>(handle);
+  Profiler& p = c->prof;
+  std::memset(out, 0, sizeof(*out));
+  for (int k = 0; k < RC_KERNEL_KINDS; ++k) {
+    out->launches[k] = p.launches[k];
+    out->flops[k] = p.flops[k];
+    out->bytes[k] = p.bytes[k];
+  }
+  for (int i = 0; i < p.used; ++i) {
+    if (cudaError_t e = cudaEventSynchronize(p.ev[2 * i + 1])) {
+      p.release();
+      return cuda_err(e, "event sync");
+    }
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, p.ev[2 * i], p.ev[2 * i + 1]);
+    out->ms[p.kind[i]] += ms;
+    out->timed[p.kind[i]]++;
+  }
+  p.release();
   return RC_OK;
 }
 
