@@ -152,6 +152,40 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
                   int frame_start, int n_frames, rc_policy policy, void* out, float* lse,
                   float* scores, int32_t* topc, int C, void* stream);
 
+/* rc_step for callers that cannot allocate device memory. The pages have no
+ * counterpart; this is a deployment convenience.
+ *
+ * rc_step keeps each call's scratch (the rotated queries of the chunk, the
+ * log-sum-exps the token scores need, and the score work buffers) inside the
+ * caller's memory block. Some callers cannot provide device memory at all:
+ * code that runs where no allocator may be called (a plugin handed a fixed
+ * budget by its host, a real-time loop that forbids allocation after start-up,
+ * a runtime whose memory accounting the library must not touch). For them this
+ * entry point places that scratch in one array inside the library's own device
+ * image instead (a file-scope __device__ array of 16 MiB, 256-byte aligned),
+ * which every GPU that loads the library holds until the process exits. It
+ * calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Arguments, layouts, results and errors are exactly those of rc_step. In
+ * addition:
+ *   - The scratch a call needs is heads * chunk_frames * frame_seqlen *
+ *     (head_dim * 2 + 4) bytes plus 8 bytes per cached token, each part
+ *     rounded up to 256 bytes; a config needing more than 16 MiB is rejected
+ *     with RC_ERANGE before anything is enqueued (e.g. 12 heads x 128 with
+ *     4680-token chunks fits; 40 heads does not).
+ *   - The first call on each device looks the array's device address up
+ *     (cudaGetSymbolAddress, with that device current) and remembers it; make
+ *     that first call before any stream capture.
+ *   - Every call, from every handle on the device, shares the one array, which
+ *     keeps the last call's contents (whatever must start at zero is cleared
+ *     by the call itself). Calls whose work overlaps on the GPU -- different
+ *     streams without ordering between them -- race on it: order them.
+ *   - The handle's own scratch region in the caller's block is not touched.
+ */
+rc_status rc_step_noalloc(void* handle, int layer, const void* q, const void* k_new,
+                          const void* v_new, int frame_start, int n_frames, rc_policy policy,
+                          void* out, float* lse, float* scores, int32_t* topc, int C, void* stream);
+
 /* Sink / time-index rewrites between chunks, applied to every layer at its
  * next new chunk: RC_REINDEX_FLUSH and/or RC_REINDEX_CUT (Infinity-RoPE),
  * RC_REINDEX_SINK (sliding / none, t_delta added to the sink's time index).

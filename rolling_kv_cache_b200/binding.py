@@ -74,7 +74,8 @@ class rc_profile(ctypes.Structure):
                 ("bytes", ctypes.c_double * 5)]
 
 
-EXPORTS = ["rc_config_init", "rc_cache_bytes", "rc_cache_create", "rc_step", "rc_reindex",
+EXPORTS = ["rc_config_init", "rc_cache_bytes", "rc_cache_create", "rc_step", "rc_step_noalloc",
+           "rc_reindex",
            "rc_get_state", "rc_device_status", "rc_rope_table", "rc_cache_layout",
            "rc_watchdog_selftest", "rc_profile_begin", "rc_profile_end", "rc_cache_destroy",
            "rc_last_error"]
@@ -94,6 +95,7 @@ def lib() -> ctypes.CDLL:
         L.rc_cache_bytes.argtypes = [ctypes.POINTER(rc_config), ctypes.POINTER(sz)]
         L.rc_cache_create.argtypes = [ctypes.POINTER(rc_config), vp, sz, ctypes.POINTER(vp)]
         L.rc_step.argtypes = [vp, i, vp, vp, vp, i, i, i, vp, vp, vp, vp, i, vp]
+        L.rc_step_noalloc.argtypes = L.rc_step.argtypes
         L.rc_reindex.argtypes = [vp, i, i, ctypes.c_uint, vp]
         L.rc_get_state.argtypes = [vp, i, ctypes.POINTER(rc_state)]
         L.rc_device_status.argtypes = [vp, vp]
@@ -140,6 +142,14 @@ def rc_step(handle, layer, q, k_new, v_new, frame_start, n_frames, policy, out, 
     check(lib().rc_step(handle, layer, q or None, k_new or None, v_new or None, frame_start,
                         n_frames, policy, out or None, lse or None, scores or None, topc or None,
                         C, stream or None))
+
+
+def rc_step_noalloc(handle, layer, q, k_new, v_new, frame_start, n_frames, policy, out, lse=0,
+                    scores=0, topc=0, C=0, stream=0) -> None:
+    """rc_step with its per-call scratch in the library's static device array."""
+    check(lib().rc_step_noalloc(handle, layer, q or None, k_new or None, v_new or None,
+                                frame_start, n_frames, policy, out or None, lse or None,
+                                scores or None, topc or None, C, stream or None))
 
 
 def rc_reindex(handle, policy, t_delta, flags, stream=0) -> None:

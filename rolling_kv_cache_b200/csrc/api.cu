@@ -466,6 +466,52 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
   return RC_OK;
 }
 
+// rc_step with its per-call scratch (rotated queries, log-sum-exps, token
+// score work buffers) placed in the library's static device array instead of
+// the caller's block: the handle's scratch pointers and query descriptor are
+// pointed there for the duration of one rc_step and restored afterwards.
+rc_status rc_step_noalloc(void* handle, int layer, const void* q, const void* k_new, const void* v_new,
+                          int frame_start, int n_frames, rc_policy policy, void* out, float* lse,
+                          float* scores, int32_t* topc, int C, void* stream) {
+  if (rc_status st = check_handle(handle)) return st;
+  Cache* c = static_cast<Cache*>(handle);
+  if (!c->device) return set_err(RC_EINVAL, "rc_step_noalloc needs a device handle");
+  const rc_config& cfg = c->cfg;
+  const MemPlan& m = c->mp;
+  const size_t q_bytes = align_up((size_t)cfg.heads * m.q_stride * cfg.head_dim * 2);
+  const size_t lse_bytes = align_up((size_t)cfg.heads * m.q_stride * 4);
+  const size_t score_bytes = align_up((size_t)m.cap * 4);
+  const size_t need = q_bytes + lse_bytes + 2 * score_bytes;
+  void* base = nullptr;
+  size_t have = 0;
+  if (cudaError_t e = rc::static_step_scratch(&base, &have)) return cuda_err(e, "static scratch lookup");
+  if (need > have)
+    return set_err(RC_ERANGE, "rc_step_noalloc needs " + std::to_string(need) +
+                                  " bytes of step scratch; the static maximum is " + std::to_string(have) +
+                                  " (heads * chunk_frames * frame_seqlen * head_dim * 2 plus scores)");
+  uint8_t* b = static_cast<uint8_t*>(base);
+  uint16_t* const saved_q = c->qrot;
+  float* const saved_lse = c->lse_scratch;
+  float* const saved_phys = c->score_phys;
+  float* const saved_logical = c->score_logical;
+  const CUtensorMap saved_map = c->tm_q;
+  const int saved_rows = c->tm_q_rows;
+  c->qrot = reinterpret_cast<uint16_t*>(b);
+  c->lse_scratch = reinterpret_cast<float*>(b + q_bytes);
+  c->score_phys = reinterpret_cast<float*>(b + q_bytes + lse_bytes);
+  c->score_logical = reinterpret_cast<float*>(b + q_bytes + lse_bytes + score_bytes);
+  c->tm_q_rows = -1;  // re-encode the query descriptor over the static array
+  const rc_status st = rc_step(handle, layer, q, k_new, v_new, frame_start, n_frames, policy, out, lse,
+                               scores, topc, C, stream);
+  c->qrot = saved_q;
+  c->lse_scratch = saved_lse;
+  c->score_phys = saved_phys;
+  c->score_logical = saved_logical;
+  c->tm_q = saved_map;
+  c->tm_q_rows = saved_rows;
+  return st;
+}
+
 rc_status rc_get_state(const void* handle, int layer, rc_state* out) {
   if (rc_status st = check_handle(handle)) return st;
   if (!out) return set_err(RC_EINVAL, "null state");

@@ -111,5 +111,8 @@ cudaError_t launch_attention(const AttnParams& p, int head_dim, cudaStream_t s);
 cudaError_t launch_scores(const ScoreParams& p, int head_dim, cudaStream_t s);
 cudaError_t launch_topc(const TopCParams& p, cudaStream_t s);
 cudaError_t launch_watchdog_selftest(int* status, unsigned limit_us, cudaStream_t s);
+// Device address and size of the static step scratch on the current device
+// (looked up once per device).
+cudaError_t static_step_scratch(void** ptr, size_t* bytes);
 
 }  // namespace rc
