@@ -71,7 +71,7 @@ def load_peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("attn_kernel.cu", "ptx.cuh", "kernels.cuh"):
+    for f in ("attn_fwd.cu", "attn_common.cuh", "ptx.cuh", "kernels.cuh"):
         with open(os.path.join(ROOT, "rolling_kv_cache_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
