@@ -262,7 +262,7 @@ rc_status rc_watchdog_selftest(void* handle, unsigned limit_us, void* stream);
  * the summed device milliseconds, then disarms. Launches beyond the limit
  * are counted but not timed. */
 enum { RC_KERNEL_REROTATE = 0, RC_KERNEL_APPEND = 1, RC_KERNEL_ATTENTION = 2,
-       RC_KERNEL_SCORES = 3, RC_KERNEL_TOPC = 4, RC_KERNEL_KINDS = 5 };
+       RC_KERNEL_SCORES = 3, RC_KERNEL_TOPC = 4, RC_KERNEL_COMBINE = 5, RC_KERNEL_KINDS = 6 };
 typedef struct rc_profile {
   int64_t launches[RC_KERNEL_KINDS];
   int64_t timed[RC_KERNEL_KINDS];

@@ -65,13 +65,13 @@ class rc_layout(ctypes.Structure):
                 ("raw_frames", ctypes.c_int32), ("total", ctypes.c_size_t)]
 
 
-RC_KERNEL_NAMES = ["rerotate", "append", "attention", "scores", "topc"]
+RC_KERNEL_NAMES = ["rerotate", "append", "attention", "scores", "topc", "combine"]
 
 
 class rc_profile(ctypes.Structure):
-    _fields_ = [("launches", ctypes.c_int64 * 5), ("timed", ctypes.c_int64 * 5),
-                ("ms", ctypes.c_double * 5), ("flops", ctypes.c_double * 5),
-                ("bytes", ctypes.c_double * 5)]
+    _fields_ = [("launches", ctypes.c_int64 * 6), ("timed", ctypes.c_int64 * 6),
+                ("ms", ctypes.c_double * 6), ("flops", ctypes.c_double * 6),
+                ("bytes", ctypes.c_double * 6)]
 
 
 EXPORTS = ["rc_config_init", "rc_cache_bytes", "rc_cache_create", "rc_step", "rc_step_noalloc",

@@ -31,9 +31,10 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct MemPlan {
-  size_t kv_bytes, raw_bytes, q_bytes, lse_bytes, score_bytes, tab_t, tab_h, tab_w, status_bytes;
+  size_t kv_bytes, raw_bytes, q_bytes, lse_bytes, score_bytes, tab_t, tab_h, tab_w, status_bytes,
+      part_o_bytes, part_lse_bytes;
   size_t off_kv, off_raw, off_q, off_lse, off_score_phys, off_score_logical, off_tab_t, off_tab_h,
-      off_tab_w, off_status, total;
+      off_tab_w, off_status, off_part_o, off_part_lse, total;
   int pt, ph, pw, cap, raw_frames, q_stride;
 };
 
@@ -56,6 +57,9 @@ MemPlan plan_memory(const rc_config& c, int raw_frames) {
   m.tab_h = align_up((size_t)c.grid_h * m.ph * 8);
   m.tab_w = align_up((size_t)c.grid_w * m.pw * 8);
   m.status_bytes = kAlign;
+  // stream-K partial rows of the attention: 2 slots per persistent CTA, 256 query rows each
+  m.part_o_bytes = align_up((size_t)2 * rc::kMaxPersistentCtas * 256 * c.head_dim * 4);
+  m.part_lse_bytes = align_up((size_t)2 * rc::kMaxPersistentCtas * 256 * 4);
   const int nraw = c.policy == RC_ROLLING_SINK ? 2 : (c.policy == RC_INFINITY_ROPE ? 1 : 0);
   size_t o = 0;
   m.off_kv = o;
@@ -78,6 +82,10 @@ MemPlan plan_memory(const rc_config& c, int raw_frames) {
   o += m.tab_w;
   m.off_status = o;
   o += m.status_bytes;
+  m.off_part_o = o;
+  o += m.part_o_bytes;
+  m.off_part_lse = o;
+  o += m.part_lse_bytes;
   m.total = o;
   return m;
 }
@@ -180,6 +188,9 @@ struct Cache {
   float* score_phys = nullptr;
   float* score_logical = nullptr;
   int* status = nullptr;
+  float* part_o = nullptr;
+  float* part_lse = nullptr;
+  int sm_count = 148;
 };
 
 rc_status check_handle(const void* h) {
@@ -256,6 +267,12 @@ rc_status rc_cache_create(const rc_config* cfg, void* dev_mem, size_t bytes, voi
     c->score_phys = reinterpret_cast<float*>(b + m.off_score_phys);
     c->score_logical = reinterpret_cast<float*>(b + m.off_score_logical);
     c->status = reinterpret_cast<int*>(b + m.off_status);
+    c->part_o = reinterpret_cast<float*>(b + m.off_part_o);
+    c->part_lse = reinterpret_cast<float*>(b + m.off_part_lse);
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+      c->sm_count = sms;
     cudaError_t e = cudaMemset(c->mem, 0, m.total);
     if (e != cudaSuccess) return cuda_err(e, "cudaMemset");
     float* tabs[3] = {reinterpret_cast<float*>(b + m.off_tab_t), reinterpret_cast<float*>(b + m.off_tab_h),
@@ -395,6 +412,31 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
   at.out = static_cast<uint16_t*>(out);
   at.lse = lse_buf;
   at.status = c->status;
+  {
+    // KV tiles each 256-query pair walks: the runs whose mask class the pair
+    // reaches, each cut into 128-token tiles (the kernels' tile walk)
+    const int NP = (Nq + 255) / 256;
+    at.n_pairs = NP;
+    if (NP <= rc::kMaxPairs) {
+      at.pair_prefix[0] = 0;
+      for (int q = 0; q < NP; ++q) {
+        const int q_last = std::min((q + 1) * 256, Nq) - 1;
+        const int rq_hi = (q_last / F) / cfg.mask_block_frames;
+        int t = 0;
+        for (const rc::Segment& g : plan.segs)
+          if (g.rank < 0 || g.rank <= rq_hi) t += (g.len + 127) / 128;
+        at.pair_prefix[q + 1] = at.pair_prefix[q] + t;
+      }
+    }
+    // persistent grid (whole-unit rounds, then stream-K over the remainder)
+    // when there are more (head, query pair) units than SMs
+    const int units = NP * H;
+    const int G = std::min(std::min(c->sm_count, rc::kMaxPersistentCtas), units);
+    const bool split = c->part_o != nullptr && units > G && NP <= rc::kMaxPairs;
+    at.part_o = split ? c->part_o : nullptr;
+    at.part_lse = split ? c->part_lse : nullptr;
+    at.n_ctas = split ? G : units;
+  }
   at.Nq = Nq;
   at.H = H;
   at.F = F;
@@ -415,8 +457,14 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
       for (int r2 = 0; r2 < n_frames; ++r2) vis += (r2 / cfg.mask_block_frames) <= (r / cfg.mask_block_frames);
       pairs += (double)F * (n_hist + (double)vis * F);
     }
-    Timed tm(c->prof, RC_KERNEL_ATTENTION, s, 4.0 * d * H * pairs, 0.0);
-    if (cudaError_t e = rc::launch_attention(at, d, s)) return cuda_err(e, "attention launch");
+    {
+      Timed tm(c->prof, RC_KERNEL_ATTENTION, s, 4.0 * d * H * pairs, 0.0);
+      if (cudaError_t e = rc::launch_attention(at, d, s)) return cuda_err(e, "attention launch");
+    }
+    if (at.part_o && (at.n_pairs * H) % at.n_ctas != 0) {
+      Timed tm(c->prof, RC_KERNEL_COMBINE, s, 0.0, (double)2 * at.n_ctas * 256 * (d + 1) * 4);
+      if (cudaError_t e = rc::launch_attention_combine(at, d, s)) return cuda_err(e, "combine launch");
+    }
   }
 
   // K6: scores over history tokens + top-C
@@ -494,8 +542,12 @@ rc_status rc_step_noalloc(void* handle, int layer, const void* q, const void* k_
   float* const saved_lse = c->lse_scratch;
   float* const saved_phys = c->score_phys;
   float* const saved_logical = c->score_logical;
+  float* const saved_part_o = c->part_o;
+  float* const saved_part_lse = c->part_lse;
   const CUtensorMap saved_map = c->tm_q;
   const int saved_rows = c->tm_q_rows;
+  c->part_o = nullptr;  // one CTA per (head, query pair): no partial rows to stage
+  c->part_lse = nullptr;
   c->qrot = reinterpret_cast<uint16_t*>(b);
   c->lse_scratch = reinterpret_cast<float*>(b + q_bytes);
   c->score_phys = reinterpret_cast<float*>(b + q_bytes + lse_bytes);
@@ -507,6 +559,8 @@ rc_status rc_step_noalloc(void* handle, int layer, const void* q, const void* k_
   c->lse_scratch = saved_lse;
   c->score_phys = saved_phys;
   c->score_logical = saved_logical;
+  c->part_o = saved_part_o;
+  c->part_lse = saved_part_lse;
   c->tm_q = saved_map;
   c->tm_q_rows = saved_rows;
   return st;

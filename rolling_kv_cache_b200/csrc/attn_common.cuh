@@ -37,6 +37,24 @@ struct TileWalker {
     }
     return false;
   }
+  // Skips the first k tiles of the walk.
+  __device__ void seek(int k) {
+    while (k > 0 && s < n_segs) {
+      const KvSegment& g = seg[s];
+      if (g.rank >= 0 && g.rank > rq_hi) {
+        ++s;
+        continue;
+      }
+      const int nt = (g.len - off + kTileRows - 1) / kTileRows;
+      if (k < nt) {
+        off += k * kTileRows;
+        return;
+      }
+      k -= nt;
+      ++s;
+      off = 0;
+    }
+  }
 };
 
 __device__ __forceinline__ int count_tiles(const KvSegment* seg, int n, int rq_hi) {

@@ -54,26 +54,111 @@ struct FwdLayout {
   static constexpr uint32_t kDynSmem = kBytes + 1024;
 };
 
+// One unit of work: query pair (rows q0 .. q0+255) of head h over the KV
+// tiles [kv_lo, kv_hi) of the pair's tile walk. slot >= 0: the job covers
+// part of its pair's tiles and leaves (O / l, log2-sum-exp) in the partial
+// workspace for the combine kernel; slot < 0: it writes the output.
+struct Job {
+  int h, q0, kv_lo, kv_hi, slot, rq_hi;
+  bool has1;
+};
+
+__device__ __forceinline__ int pair_rq_hi(const AttnParams& p, int pair) {
+  const int q_last = min((pair + 1) * 2 * kTileRows, p.Nq) - 1;
+  return (q_last / p.F) / p.mask_block;
+}
+
+// Persistent schedule over units u = h * NP + pair (head-major), each with
+// T(pair) KV tiles (pair_prefix). Rounds first: CTA c takes whole units
+// c, c + G, ... for R = U / G rounds; the G CTAs of a round all start at KV
+// tile 0 together, so the query pairs of a head read each K/V tile about
+// when the others do and it comes from DRAM once. The U mod G units left
+// over (the last heads) are then cut stream-K style: their tiles, in (unit,
+// tile) order, are split into G equal ranges, one per CTA; a unit cut
+// between CTAs leaves partial rows for the combine kernel. Their K/V spans
+// only a few heads, so it stays in L2 whatever the offsets.
+// Without a partial workspace the grid has one CTA per unit.
+struct Scheduler {
+  const AttnParams* p;
+  int NP, T_head, c, G, rounds, r;
+  long long pos, end, base;
+  bool split, first_sk;
+
+  __device__ long long cum(long long u) const {  // tiles of units [0, u)
+    return (u / NP) * T_head + p->pair_prefix[u % NP];
+  }
+
+  __device__ void init(const AttnParams& prm) {
+    p = &prm;
+    NP = prm.n_pairs;
+    c = blockIdx.x;
+    G = gridDim.x;
+    split = prm.part_o != nullptr;
+    T_head = split ? prm.pair_prefix[NP] : 0;  // the prefix table is filled for persistent launches
+    first_sk = true;
+    r = 0;
+    const long long U = (long long)NP * prm.H;
+    rounds = split ? (int)(U / G) : 1;
+    pos = end = 0;
+    if (split) {
+      base = cum((long long)rounds * G);
+      const long long W_rem = cum(U) - base;
+      pos = base + (long long)c * W_rem / G;
+      end = base + (long long)(c + 1) * W_rem / G;
+    }
+  }
+
+  __device__ void fill(Job& j, int h, int pair, int off, int len, int T_u, int slot) const {
+    j.h = h;
+    j.q0 = pair * 2 * kTileRows;
+    j.kv_lo = off;
+    j.kv_hi = off + len;
+    j.rq_hi = pair_rq_hi(*p, pair);
+    j.has1 = j.q0 + kTileRows < p->Nq;
+    j.slot = (off > 0 || off + len < T_u) ? slot : -1;
+  }
+
+  __device__ bool next(Job& j) {
+    if (r < rounds) {
+      const int u = c + r * G;
+      ++r;
+      const int pair = u % NP;
+      const int T_u = split ? p->pair_prefix[pair + 1] - p->pair_prefix[pair]
+                            : count_tiles(p->seg, p->n_segs, pair_rq_hi(*p, pair));
+      fill(j, u / NP, pair, 0, T_u, T_u, -1);
+      return true;
+    }
+    if (pos >= end) return false;
+    const int h = (int)(pos / T_head);
+    const int rem = (int)(pos - (long long)h * T_head);
+    int pair = 0;
+    while (p->pair_prefix[pair + 1] <= rem) ++pair;
+    const int T_u = p->pair_prefix[pair + 1] - p->pair_prefix[pair];
+    const int off = rem - p->pair_prefix[pair];
+    const int len = (int)min((long long)(T_u - off), end - pos);
+    pos += len;
+    fill(j, h, pair, off, len, T_u, 2 * c + (first_sk ? 0 : 1));
+    first_sk = false;
+    return true;
+  }
+};
+
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
   using L = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_q, bar_kf[2], bar_vf[2], bar_ke[2], bar_ve[2], bar_s[2], bar_p[2], bar_o[2], bar_fin;
+  __shared__ uint64_t bar_q, bar_qe, bar_kf[2], bar_vf[2], bar_ke[2], bar_ve[2], bar_s[2], bar_p[2], bar_o[2],
+      bar_fin;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.y;
-  const int q0 = blockIdx.x * 2 * kTileRows;
-  const bool has1 = q0 + kTileRows < p.Nq;
-  const int q_last = min(q0 + 2 * kTileRows, p.Nq) - 1;
-  const int rq_hi = (q_last / p.F) / p.mask_block;
-  const int T = count_tiles(p.seg, p.n_segs, rq_hi);
   const uint32_t base_u32 = (ptx::smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_u32 - ptx::smem_u32(smem_raw));
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&bar_q, 1);
+    ptx::mbar_init(&bar_qe, 1);
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&bar_kf[i], 1);
       ptx::mbar_init(&bar_vf[i], 1);
@@ -96,40 +181,50 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   ptx::tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
   volatile int* abort = &abort_sh;
+  int dummy_abort = 0;
+  volatile int* noabort = reinterpret_cast<volatile int*>(&dummy_abort);
+  Scheduler sc;
+  sc.init(p);
+  Job jb;
 
   if (warp == kProducerWarp && lane == 0) {
     // ---------------------------------------------------------- producer
     ptx::tma_prefetch_desc(&p.tm_q);
     ptx::tma_prefetch_desc(&p.tm_k);
     ptx::tma_prefetch_desc(&p.tm_v);
-    ptx::mbar_arrive_expect_tx(&bar_q, (has1 ? 2 : 1) * L::kTile);
-    for (int i = 0; i < (has1 ? 2 : 1); ++i)
-      for (int j = 0; j < L::kSub; ++j)
-        ptx::tma_load_3d(&p.tm_q, &bar_q, base + L::kQ + i * L::kTile + j * kSubTileBytes, 64 * j,
-                         q0 + i * kTileRows, h);
-    TileWalker wk{p.seg, p.n_segs, rq_hi};
-    Tile t;
+    int nq = 0, g = 0;
     int nk[2] = {0, 0}, nv[2] = {0, 0};  // loads issued per stage
-    for (int it = 0; wk.next(t); ++it) {
-      const int st = it & 1;
-      const uint32_t free_par = ((it >> 1) - 1) & 1;
-      if (it >= 2 && !ptx::mbar_wait(&bar_ke[st], free_par, abort, p.status, RC_ETIMEOUT)) break;
-      ptx::mbar_arrive_expect_tx(&bar_kf[st], L::kTile);
-      for (int j = 0; j < L::kSub; ++j)
-        ptx::tma_load_3d(&p.tm_k, &bar_kf[st], base + L::kK + st * L::kTile + j * kSubTileBytes, 64 * j,
-                         t.tok, h);
-      nk[st]++;
-      if (it >= 2 && !ptx::mbar_wait(&bar_ve[st], free_par, abort, p.status, RC_ETIMEOUT)) break;
-      ptx::mbar_arrive_expect_tx(&bar_vf[st], L::kTile);
-      for (int j = 0; j < L::kSub; ++j)
-        ptx::tma_load_3d(&p.tm_v, &bar_vf[st], base + L::kV + st * L::kTile + j * kSubTileBytes, 64 * j,
-                         t.tok, h);
-      nv[st]++;
+    bool ok = true;
+    while (ok && sc.next(jb)) {
+      if (nq > 0 && !ptx::mbar_wait(&bar_qe, (nq - 1) & 1, abort, p.status, RC_ETIMEOUT)) break;
+      ptx::mbar_arrive_expect_tx(&bar_q, (jb.has1 ? 2 : 1) * L::kTile);
+      for (int i = 0; i < (jb.has1 ? 2 : 1); ++i)
+        for (int j = 0; j < L::kSub; ++j)
+          ptx::tma_load_3d(&p.tm_q, &bar_q, base + L::kQ + i * L::kTile + j * kSubTileBytes, 64 * j,
+                           jb.q0 + i * kTileRows, jb.h);
+      ++nq;
+      TileWalker wk{p.seg, p.n_segs, jb.rq_hi};
+      wk.seek(jb.kv_lo);
+      Tile t;
+      for (int j = jb.kv_lo; j < jb.kv_hi && wk.next(t); ++j, ++g) {
+        const int st = g & 1;
+        const uint32_t free_par = ((g >> 1) - 1) & 1;
+        if (g >= 2 && !ptx::mbar_wait(&bar_ke[st], free_par, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
+        ptx::mbar_arrive_expect_tx(&bar_kf[st], L::kTile);
+        for (int k = 0; k < L::kSub; ++k)
+          ptx::tma_load_3d(&p.tm_k, &bar_kf[st], base + L::kK + st * L::kTile + k * kSubTileBytes, 64 * k,
+                           t.tok, jb.h);
+        nk[st]++;
+        if (g >= 2 && !ptx::mbar_wait(&bar_ve[st], free_par, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
+        ptx::mbar_arrive_expect_tx(&bar_vf[st], L::kTile);
+        for (int k = 0; k < L::kSub; ++k)
+          ptx::tma_load_3d(&p.tm_v, &bar_vf[st], base + L::kV + st * L::kTile + k * kSubTileBytes, 64 * k,
+                           t.tok, jb.h);
+        nv[st]++;
+      }
     }
     // never leave a copy in flight: wait (bounded, ignoring abort) for the last ones
-    int dummy = 0;
-    volatile int* noabort = reinterpret_cast<volatile int*>(&dummy);
-    ptx::mbar_wait(&bar_q, 0, noabort, p.status, RC_ETIMEOUT);
+    if (nq) ptx::mbar_wait(&bar_q, (nq - 1) & 1, noabort, p.status, RC_ETIMEOUT);
     for (int st = 0; st < 2; ++st) {
       if (nk[st]) ptx::mbar_wait(&bar_kf[st], (nk[st] - 1) & 1, noabort, p.status, RC_ETIMEOUT);
       if (nv[st]) ptx::mbar_wait(&bar_vf[st], (nv[st] - 1) & 1, noabort, p.status, RC_ETIMEOUT);
@@ -158,167 +253,199 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
                     ptx::sdesc_sw128(sV + ks * 2048, kSubTileBytes, 1024), idesc_o, acc || ks > 0);
       ptx::mma_commit(&bar_o[i]);
     };
-    bool ok = ptx::mbar_wait(&bar_q, 0, abort, p.status, RC_ETIMEOUT);
-    if (ok && T > 0) {
-      ok = ptx::mbar_wait(&bar_kf[0], 0, abort, p.status, RC_ETIMEOUT);
-      if (ok) {
-        ptx::tc_fence_after();
-        issue_s(0, 0);
-        if (has1) issue_s(1, 0);
-        ptx::mma_commit(&bar_ke[0]);
-      }
-    }
-    for (int j = 0; ok && j < T; ++j) {
-      const int st = j & 1, st1 = (j + 1) & 1;
-      const uint32_t par = j & 1;
-      if (!ptx::mbar_wait(&bar_p[0], par, abort, p.status, RC_ETIMEOUT)) break;
-      if (!ptx::mbar_wait(&bar_vf[st], (j >> 1) & 1, abort, p.status, RC_ETIMEOUT)) break;
+    int nq = 0, g = 0, gp[2] = {0, 0};
+    bool ok = true;
+    while (ok && sc.next(jb)) {
+      const int n = jb.kv_hi - jb.kv_lo;
+      const bool two = jb.has1;
+      if (!ptx::mbar_wait(&bar_q, nq & 1, abort, p.status, RC_ETIMEOUT)) break;
+      ++nq;
+      if (!ptx::mbar_wait(&bar_kf[g & 1], (g >> 1) & 1, abort, p.status, RC_ETIMEOUT)) break;
       ptx::tc_fence_after();
-      issue_pv(0, st, j > 0);
-      if (!has1) ptx::mma_commit(&bar_ve[st]);
-      const bool more = j + 1 < T;
-      if (more) {
-        if (!ptx::mbar_wait(&bar_kf[st1], ((j + 1) >> 1) & 1, abort, p.status, RC_ETIMEOUT)) break;
+      issue_s(0, g & 1);
+      if (two) issue_s(1, g & 1);
+      ptx::mma_commit(&bar_ke[g & 1]);
+      if (n == 1) ptx::mma_commit(&bar_qe);
+      for (int j = 0; j < n; ++j, ++g) {
+        const int st = g & 1, st1 = (g + 1) & 1;
+        const bool more = j + 1 < n;
+        if (!ptx::mbar_wait(&bar_p[0], gp[0] & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
+        if (!ptx::mbar_wait(&bar_vf[st], (g >> 1) & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
         ptx::tc_fence_after();
-        issue_s(0, st1);
-        if (!has1) ptx::mma_commit(&bar_ke[st1]);
-      }
-      if (has1) {
-        if (!ptx::mbar_wait(&bar_p[1], par, abort, p.status, RC_ETIMEOUT)) break;
-        ptx::tc_fence_after();
-        issue_pv(1, st, j > 0);
-        ptx::mma_commit(&bar_ve[st]);
+        issue_pv(0, st, j > 0);
+        ++gp[0];
+        if (!two) ptx::mma_commit(&bar_ve[st]);
         if (more) {
-          issue_s(1, st1);
-          ptx::mma_commit(&bar_ke[st1]);
+          if (!ptx::mbar_wait(&bar_kf[st1], ((g + 1) >> 1) & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
+          ptx::tc_fence_after();
+          issue_s(0, st1);
+          if (!two) {
+            ptx::mma_commit(&bar_ke[st1]);
+            if (j + 2 == n) ptx::mma_commit(&bar_qe);
+          }
+        }
+        if (two) {
+          if (!ptx::mbar_wait(&bar_p[1], gp[1] & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
+          ptx::tc_fence_after();
+          issue_pv(1, st, j > 0);
+          ++gp[1];
+          ptx::mma_commit(&bar_ve[st]);
+          if (more) {
+            issue_s(1, st1);
+            ptx::mma_commit(&bar_ke[st1]);
+            if (j + 2 == n) ptx::mma_commit(&bar_qe);
+          }
         }
       }
     }
-    int dummy = 0;
     ptx::mma_commit(&bar_fin);
-    ptx::mbar_wait(&bar_fin, 0, reinterpret_cast<volatile int*>(&dummy), p.status, RC_ETIMEOUT);
-  } else if (warp < 8 && (warp < 4 || has1)) {
+    ptx::mbar_wait(&bar_fin, 0, noabort, p.status, RC_ETIMEOUT);
+  } else if (warp < 8) {
     // ---------------------------------------------------------- softmax
     const int grp = warp >> 2;
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
-    const int qtok = q0 + grp * kTileRows + row;
-    const int my_rank = (min(qtok, p.Nq - 1) / p.F) / p.mask_block;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + grp * 128;
     const uint32_t tO = tmem + lane_off + 256 + grp * 128;
     const float c = p.scale_log2;
     const float thresh = kRescaleLog2 / c;
-    float m = -INFINITY, l = 0.f;
-    TileWalker wk{p.seg, p.n_segs, rq_hi};
-    Tile t;
-    bool ok = true;
-    for (int j = 0; wk.next(t); ++j) {
-      if (!ptx::mbar_wait(&bar_s[grp], j & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
-      ptx::tc_fence_after();
-      // columns [0, lim) of this row are visible (the whole row or a ragged tail is masked)
-      const int lim = (t.rank < 0 || t.rank <= my_rank) ? t.nvalid : 0;
-      // pass 1: row maximum of the raw scores
-      float mx = -INFINITY;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t r[32];
-        ptx::tmem_ld32(tS + cc * 32, r);
-        ptx::tmem_ld_wait();
-        if (lim == kTileRows) {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) mx = fmaxf(mx, __uint_as_float(r[k]));
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) mx = fmaxf(mx, cc * 32 + k < lim ? __uint_as_float(r[k]) : -INFINITY);
-        }
-      }
-      const float m_new = fmaxf(m, mx);
-      const bool need = m_new > m + thresh;       // also true for the first visible tile
-      const bool real = need && m != -INFINITY;   // O already holds weighted values
-      if (__any_sync(0xffffffffu, real)) {
-        if (!ptx::mbar_wait(&bar_o[grp], (j - 1) & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
+    int gs = 0;  // this group's tiles so far (phase of bar_s / bar_p / bar_o)
+    while (sc.next(jb)) {
+      if (*abort) break;
+      if (grp == 1 && !jb.has1) continue;
+      const int qtok = jb.q0 + grp * kTileRows + row;
+      const int my_rank = (min(qtok, p.Nq - 1) / p.F) / p.mask_block;
+      float m = -INFINITY, l = 0.f;
+      TileWalker wk{p.seg, p.n_segs, jb.rq_hi};
+      wk.seek(jb.kv_lo);
+      Tile t;
+      bool ok = true;
+      int done = 0;
+      for (int j = jb.kv_lo; j < jb.kv_hi && wk.next(t); ++j) {
+        if (!ptx::mbar_wait(&bar_s[grp], gs & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
         ptx::tc_fence_after();
-        const float alpha = real ? ptx::ex2((m - m_new) * c) : 1.f;
+        // columns [0, lim) of this row are visible (the whole row or a ragged tail is masked)
+        const int lim = (t.rank < 0 || t.rank <= my_rank) ? t.nvalid : 0;
+        // pass 1: row maximum of the raw scores
+        float mx = -INFINITY;
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          ptx::tmem_ld32(tO + cc * 32, o);
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t r[32];
+          ptx::tmem_ld32(tS + cc * 32, r);
           ptx::tmem_ld_wait();
+          if (lim == kTileRows) {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          ptx::tmem_st32(tO + cc * 32, o);
+            for (int k = 0; k < 32; ++k) mx = fmaxf(mx, __uint_as_float(r[k]));
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) mx = fmaxf(mx, cc * 32 + k < lim ? __uint_as_float(r[k]) : -INFINITY);
+          }
+        }
+        const float m_new = fmaxf(m, mx);
+        const bool need = m_new > m + thresh;       // also true for the first visible tile
+        const bool real = need && m != -INFINITY;   // O already holds weighted values
+        if (__any_sync(0xffffffffu, real)) {
+          if (!ptx::mbar_wait(&bar_o[grp], (gs - 1) & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
+          ptx::tc_fence_after();
+          const float alpha = real ? ptx::ex2((m - m_new) * c) : 1.f;
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            ptx::tmem_ld32(tO + cc * 32, o);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            ptx::tmem_st32(tO + cc * 32, o);
+          }
+          ptx::tmem_st_wait();
+          l *= alpha;
+        }
+        if (need) m = m_new;
+        const float mc = (m == -INFINITY ? 0.f : m) * c;
+        // pass 2: P = 2^(s c - m c), packed bf16 pairs written over S's first
+        // 64 columns; chunk cc's P columns [16cc, 16cc+16) lie in S columns
+        // already read, so the overwrite never races a later read.
+        float sum = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t r[32];
+          ptx::tmem_ld32(tS + cc * 32, r);
+          ptx::tmem_ld_wait();
+          uint32_t pk[16];
+          if (lim == kTileRows) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const float a = ptx::ex2(fmaf(__uint_as_float(r[2 * k]), c, -mc));
+              const float b = ptx::ex2(fmaf(__uint_as_float(r[2 * k + 1]), c, -mc));
+              sum += a + b;
+              pk[k] = ptx::pack_bf16x2(a, b);
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const float a = cc * 32 + 2 * k < lim ? ptx::ex2(fmaf(__uint_as_float(r[2 * k]), c, -mc)) : 0.f;
+              const float b =
+                  cc * 32 + 2 * k + 1 < lim ? ptx::ex2(fmaf(__uint_as_float(r[2 * k + 1]), c, -mc)) : 0.f;
+              sum += a + b;
+              pk[k] = ptx::pack_bf16x2(a, b);
+            }
+          }
+          ptx::tmem_st16(tS + cc * 16, pk);
         }
         ptx::tmem_st_wait();
-        l *= alpha;
+        l += sum;
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bar_p[grp]);
+        ++gs;
+        ++done;
       }
-      if (need) m = m_new;
-      const float mc = (m == -INFINITY ? 0.f : m) * c;
-      // pass 2: P = 2^(s c - m c), packed bf16 pairs written over S's first
-      // 64 columns; chunk cc's P columns [16cc, 16cc+16) lie in S columns
-      // already read, so the overwrite never races a later read.
-      float sum = 0.f;
+      // epilogue: O / l, to the output (bf16 [Nq][H][D], lse in natural log)
+      // or to this CTA's partial slot (fp32, log2-sum-exp)
+      const bool have_o =
+          ok && done > 0 && ptx::mbar_wait(&bar_o[grp], (gs - 1) & 1, abort, p.status, RC_ETIMEOUT);
+      ptx::tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float lse2 = l > 0.f ? m * c + __log2f(l) : -INFINITY;
+      const int prow = grp * kTileRows + row;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t r[32];
-        ptx::tmem_ld32(tS + cc * 32, r);
-        ptx::tmem_ld_wait();
-        uint32_t pk[16];
-        if (lim == kTileRows) {
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float a = ptx::ex2(fmaf(__uint_as_float(r[2 * k]), c, -mc));
-            const float b = ptx::ex2(fmaf(__uint_as_float(r[2 * k + 1]), c, -mc));
-            sum += a + b;
-            pk[k] = ptx::pack_bf16x2(a, b);
-          }
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        if (have_o) {
+          ptx::tmem_ld32(tO + cc * 32, o);
+          ptx::tmem_ld_wait();
         } else {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float a = cc * 32 + 2 * k < lim ? ptx::ex2(fmaf(__uint_as_float(r[2 * k]), c, -mc)) : 0.f;
-            const float b = cc * 32 + 2 * k + 1 < lim ? ptx::ex2(fmaf(__uint_as_float(r[2 * k + 1]), c, -mc)) : 0.f;
-            sum += a + b;
-            pk[k] = ptx::pack_bf16x2(a, b);
-          }
+          for (int k = 0; k < 32; ++k) o[k] = 0u;
         }
-        ptx::tmem_st16(tS + cc * 16, pk);
-      }
-      ptx::tmem_st_wait();
-      l += sum;
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bar_p[grp]);
-    }
-    // epilogue: O / l -> bf16 [Nq][H][D]; lse in natural log
-    const int T_done = ok ? T : 0;
-    bool have_o = T_done > 0 && ptx::mbar_wait(&bar_o[grp], (T_done - 1) & 1, abort, p.status, RC_ETIMEOUT);
-    ptx::tc_fence_after();
-    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+        if (qtok >= p.Nq) continue;
+        if (jb.slot < 0) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)qtok * p.H + jb.h) * D + cc * 32);
 #pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
-      uint32_t o[32];
-      if (have_o) {
-        ptx::tmem_ld32(tO + cc * 32, o);
-        ptx::tmem_ld_wait();
-      } else {
+          for (int v = 0; v < 4; ++v) {
+            uint4 u;
+            u.x = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
+            u.y = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
+            u.z = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
+            u.w = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
+            dst[v] = u;
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(p.part_o + ((size_t)jb.slot * 2 * kTileRows + prow) * D + cc * 32);
 #pragma unroll
-        for (int k = 0; k < 32; ++k) o[k] = 0u;
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
+                                 __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
+        }
       }
       if (qtok < p.Nq) {
-        uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)qtok * p.H + h) * D + cc * 32);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint4 u;
-          u.x = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
-          u.y = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
-          u.z = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
-          u.w = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
-          dst[v] = u;
+        if (jb.slot < 0) {
+          if (p.lse) p.lse[(size_t)jb.h * p.Nq + qtok] = lse2 * 0.69314718055994531f;
+        } else {
+          p.part_lse[(size_t)jb.slot * 2 * kTileRows + prow] = lse2;
         }
       }
-    }
-    if (p.lse && qtok < p.Nq) {
-      const float lse2 = l > 0.f ? m * c + __log2f(l) : -INFINITY;
-      p.lse[(size_t)h * p.Nq + qtok] = lse2 * 0.69314718055994531f;
+      if (!ok) break;
     }
   }
   ptx::tc_fence_before();
@@ -327,6 +454,84 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, 512);
   }
+}
+
+// K5: merges the partial results of the (head, pair) units the stream-K
+// schedule split between CTAs: O = sum_i 2^(lse_i - lse) O_i with
+// lse = log2 sum_i 2^(lse_i). Block (unit, y) takes 32 query rows of the
+// unit; 8 consecutive threads share a row, D/8 columns each, so every warp
+// reads 4 whole rows of a partial at once.
+__device__ __forceinline__ long long owner_of(long long pos, long long W, int G) {
+  return ((pos + 1) * G - 1) / W;  // largest c with floor(c W / G) <= pos
+}
+
+constexpr int kCombineRowsPerBlock = 32;
+
+template <int D>
+__global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant__ AttnParams p, int G) {
+  constexpr int kCols = D / 8;
+  const int NP = p.n_pairs;
+  const long long T_head = p.pair_prefix[NP];
+  const long long U = (long long)NP * p.H;
+  const long long first_rem = (U / G) * G;  // units before it ran in whole-unit rounds
+  const long long u = first_rem + blockIdx.x;
+  if (u >= U) return;
+  const int h = (int)(u / NP), pair = (int)(u % NP);
+  auto cum = [&](long long v) { return (v / NP) * T_head + p.pair_prefix[v % NP]; };
+  const long long base = cum(first_rem);
+  const long long W = cum(U) - base;
+  const long long C_u = cum(u) - base;  // unit start in the stream-K range
+  const int T_u = p.pair_prefix[pair + 1] - p.pair_prefix[pair];
+  const int c_lo = (int)owner_of(C_u, W, G), c_hi = (int)owner_of(C_u + T_u - 1, W, G);
+  if (c_lo == c_hi) return;  // written directly by one CTA
+  const int prow = blockIdx.y * kCombineRowsPerBlock + (threadIdx.x >> 3);
+  const int col0 = (threadIdx.x & 7) * kCols;
+  const int qtok = pair * 2 * kTileRows + prow;
+  if (qtok >= p.Nq) return;
+  // slot of CTA c's job on this unit: its first job iff its range starts inside the unit
+  auto slot_of = [&](int cc) {
+    const long long b = (long long)cc * W / G;
+    return 2 * cc + ((b >= C_u) ? 0 : 1);
+  };
+  // a CTA whose stream-K range is empty (fewer remainder tiles than CTAs) holds no part
+  auto has_part = [&](int cc) { return (long long)(cc + 1) * W / G > (long long)cc * W / G; };
+  float mx = -INFINITY;
+  for (int cc = c_lo; cc <= c_hi; ++cc)
+    if (has_part(cc)) mx = fmaxf(mx, p.part_lse[(size_t)slot_of(cc) * 2 * kTileRows + prow]);
+  float acc[kCols];
+#pragma unroll
+  for (int k = 0; k < kCols; ++k) acc[k] = 0.f;
+  float den = 0.f;
+  for (int cc = c_lo; cc <= c_hi; ++cc) {
+    if (!has_part(cc)) continue;
+    const int sl = slot_of(cc);
+    const float ls = p.part_lse[(size_t)sl * 2 * kTileRows + prow];
+    const float w = ls == -INFINITY ? 0.f : exp2f(ls - mx);
+    den += w;
+    const float4* src =
+        reinterpret_cast<const float4*>(p.part_o + ((size_t)sl * 2 * kTileRows + prow) * D + col0);
+#pragma unroll
+    for (int v = 0; v < kCols / 4; ++v) {
+      const float4 x = src[v];
+      acc[4 * v] += w * x.x;
+      acc[4 * v + 1] += w * x.y;
+      acc[4 * v + 2] += w * x.z;
+      acc[4 * v + 3] += w * x.w;
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)qtok * p.H + h) * D + col0);
+#pragma unroll
+  for (int v = 0; v < kCols / 8; ++v) {
+    uint4 x;
+    x.x = ptx::pack_bf16x2(acc[8 * v] * inv, acc[8 * v + 1] * inv);
+    x.y = ptx::pack_bf16x2(acc[8 * v + 2] * inv, acc[8 * v + 3] * inv);
+    x.z = ptx::pack_bf16x2(acc[8 * v + 4] * inv, acc[8 * v + 5] * inv);
+    x.w = ptx::pack_bf16x2(acc[8 * v + 6] * inv, acc[8 * v + 7] * inv);
+    dst[v] = x;
+  }
+  if (p.lse && (threadIdx.x & 7) == 0)
+    p.lse[(size_t)h * p.Nq + qtok] = (den > 0.f ? mx + log2f(den) : -INFINITY) * 0.69314718055994531f;
 }
 
 template <int D>
@@ -339,16 +544,28 @@ cudaError_t launch_fwd_d(const AttnParams& p, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid((p.Nq + 2 * kTileRows - 1) / (2 * kTileRows), p.H);
-  attn_fwd_kernel<D><<<grid, kFwdThreads, L::kDynSmem, s>>>(p);
+  attn_fwd_kernel<D><<<p.n_ctas, kFwdThreads, L::kDynSmem, s>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attention(const AttnParams& p, int head_dim, cudaStream_t s) {
-  if (p.Nq <= 0) return cudaSuccess;
+  if (p.Nq <= 0 || p.n_ctas <= 0) return cudaSuccess;
   return head_dim == 64 ? launch_fwd_d<64>(p, s) : launch_fwd_d<128>(p, s);
+}
+
+cudaError_t launch_attention_combine(const AttnParams& p, int head_dim, cudaStream_t s) {
+  if (p.Nq <= 0 || !p.part_o) return cudaSuccess;
+  const int units = p.n_pairs * p.H;
+  const int rem = units % p.n_ctas;  // units of the stream-K remainder
+  if (rem == 0) return cudaSuccess;
+  const dim3 grid(rem, 2 * kTileRows / kCombineRowsPerBlock);
+  if (head_dim == 64)
+    attn_combine_kernel<64><<<grid, 256, 0, s>>>(p, p.n_ctas);
+  else
+    attn_combine_kernel<128><<<grid, 256, 0, s>>>(p, p.n_ctas);
+  return cudaGetLastError();
 }
 
 }  // namespace rc

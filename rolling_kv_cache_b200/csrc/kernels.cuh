@@ -14,6 +14,11 @@ namespace rc {
 constexpr int kMaxJobs = 64;
 constexpr int kMaxSegs = 48;  // == kEngineMaxSegs
 constexpr int kMaxCandFrames = RC_MAX_SLOTS;
+// Most CTAs a persistent attention launch uses (>= the B200's 148 SMs); sizes
+// the partial-result workspace: 2 slots per CTA.
+constexpr int kMaxPersistentCtas = 160;
+// Most 256-query pairs a persistent attention launch schedules (per head).
+constexpr int kMaxPairs = 128;
 
 struct RopeTables {
   const float2* t;  // [t_max][pt]   (cos, sin)
@@ -76,10 +81,15 @@ struct alignas(64) AttnParams {
   uint16_t* out;       // [Nq][H][d] bf16
   float* lse;          // [H][Nq] or null
   int* status;         // device status word
+  float* part_o;       // null, or stream-K partials [2 * n_ctas][256][d] fp32 (O / l)
+  float* part_lse;     // [2 * n_ctas][256] fp32, log2-sum-exp of each partial row
+  int n_ctas;          // grid size: persistent CTAs (with partials) or one per (head, pair)
   int Nq, H, F, mask_block;
   float scale_log2;    // log2(e) / sqrt(d)
   int n_segs;
   KvSegment seg[kMaxSegs];
+  int n_pairs;                      // query pairs per head (persistent launches)
+  int pair_prefix[kMaxPairs + 1];   // KV tiles of pairs [0, q) (same for every head)
 };
 
 // K6a: column scores over history tokens (second QK^T pass with final LSE).
@@ -108,6 +118,8 @@ struct TopCParams {
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t launch_rerotate(const RerotateParams& p, cudaStream_t s);
 cudaError_t launch_attention(const AttnParams& p, int head_dim, cudaStream_t s);
+// K5: merges the partial rows of split (head, pair) units; only after a launch with partials.
+cudaError_t launch_attention_combine(const AttnParams& p, int head_dim, cudaStream_t s);
 cudaError_t launch_scores(const ScoreParams& p, int head_dim, cudaStream_t s);
 cudaError_t launch_topc(const TopCParams& p, cudaStream_t s);
 cudaError_t launch_watchdog_selftest(int* status, unsigned limit_us, cudaStream_t s);
