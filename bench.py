@@ -137,6 +137,23 @@ class ClockSampler:
                 "samples": len(self.rows)}
 
 
+def aggregate_over_ranks(ms: float, work: float, device=None):
+    """(max of ms, sum of work) over the ranks of the default process group.
+
+    Whole-job throughput = summed work over the slowest rank's time. With a
+    single process it returns its inputs. Every rank calls it at the same
+    point (same collectives, same order)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms, work
+    t_max = torch.tensor([ms], dtype=torch.float64, device=device)
+    t_sum = torch.tensor([work], dtype=torch.float64, device=device)
+    dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    dist.all_reduce(t_sum, op=dist.ReduceOp.SUM)
+    return float(t_max[0]), float(t_sum[0])
+
+
 def make_cfg(w, layers=None):
     from rolling_kv_cache_b200.cache import make_config
     return make_config(layers=w.layers if layers is None else layers, heads=w.heads,
@@ -262,15 +279,7 @@ def run_ours(args, w):
     cache.device_status()
 
     att = prof["attention"]
-    flops_rank = att["flops"]
-    ms_max = ms
-    flops_total = flops_rank
-    if world > 1:
-        t = torch.tensor([ms, flops_rank], dtype=torch.float64, device=dev)
-        mx = t.clone()
-        dist.all_reduce(mx[:1], op=dist.ReduceOp.MAX)
-        dist.all_reduce(t[1:], op=dist.ReduceOp.SUM)
-        ms_max, flops_total = float(mx[0]), float(t[1])
+    ms_max, flops_total = aggregate_over_ranks(ms, att["flops"], dev)
     value = flops_total / (ms_max / 1e3) / 1e12
     frames = args.steps * B_ * world
     frames_per_s_per_layer = frames / (ms_max / 1e3) * w.layers / world
@@ -295,14 +304,7 @@ def run_ours(args, w):
         chunk += 1
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    e2e_tot = e2e_flops
-    if world > 1:
-        t = torch.tensor([e2e_ms, e2e_flops], dtype=torch.float64, device=dev)
-        mx = t.clone()
-        dist.all_reduce(mx[:1], op=dist.ReduceOp.MAX)
-        dist.all_reduce(t[1:], op=dist.ReduceOp.SUM)
-        e2e_ms, e2e_tot = float(mx[0]), float(t[1])
+    e2e_ms, e2e_tot = aggregate_over_ranks(e0.elapsed_time(e1), e2e_flops, dev)
     e2e_value = e2e_tot / (e2e_ms / 1e3) / 1e12
 
     peaks, peak_src = load_peaks()
