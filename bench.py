@@ -240,12 +240,18 @@ def run_ours(args, w):
     out = torch.empty_like(pool[0][0])
     B_ = w.chunk_frames
     calls_per_step = w.layers * w.passes
+    # Deep-Forcing token scores + top-C on every step where the workload asks for them
+    scores = torch.empty(w.footprint_tokens, dtype=torch.float32, device=dev) if w.topc else None
+    topc = torch.empty(w.topc, dtype=torch.int32, device=dev) if w.topc else None
 
-    def run_chunk(c):
+    def run_chunk(c, q_of=None, out_buf=None):
+        if c in w.cut_chunks:   # KV flush + RoPE cut before the chunk's first pass
+            cache.reindex(w.cut_delta, B.RC_REINDEX_FLUSH | B.RC_REINDEX_CUT)
         for p in range(w.passes):
             for l in range(w.layers):
-                q, k, v = pool[(c * 7 + p * 3 + l) % len(pool)]
-                cache.step(l, q, k, v, c * B_, out=out)
+                q, k, v = (q_of or pool)[(c * 7 + p * 3 + l) % len(q_of or pool)]
+                cache.step(l, q, k, v, c * B_, out=out if out_buf is None else out_buf,
+                           scores=scores, topc=topc, C=w.topc)
 
     chunk = 0
     prefill = (w.footprint_frames + B_ - 1) // B_   # until the window is full
@@ -259,7 +265,7 @@ def run_ours(args, w):
     if world > 1:
         dist.barrier()
 
-    B.rc_profile_begin(cache.handle, args.steps * calls_per_step * 2 + 16)
+    B.rc_profile_begin(cache.handle, args.steps * calls_per_step * 6 + 16)
     gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
     if not gpu_uuid.startswith("GPU-"):
         gpu_uuid = "GPU-" + gpu_uuid
@@ -288,21 +294,26 @@ def run_ours(args, w):
     # ---------------- end to end through the public API with host buffers
     e2e_steps = max(1, args.e2e_steps)
     host_pool = [tuple(t.cpu().pin_memory() for t in trip) for trip in pool[:3]]
-    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    out_hosts = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
     h2d = sum(t.numel() * 2 for t in host_pool[0]) * calls_per_step
-    d2h = out_host.numel() * 2 * calls_per_step
+    d2h = out_hosts[0].numel() * 2 * calls_per_step
+    pipe = cache.host_pipeline(depth=2)
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     e2e_flops = 0.0
     for _ in range(e2e_steps):
+        if chunk in w.cut_chunks:
+            cache.reindex(w.cut_delta, B.RC_REINDEX_FLUSH | B.RC_REINDEX_CUT)
         for p in range(w.passes):
             for l in range(w.layers):
                 q, k, v = host_pool[(p + l) % len(host_pool)]
-                cache.step(l, q, k, v, chunk * B_, out=out_host)
-        e2e_flops += attention_flops(w, steady_hist_frames(w)) * calls_per_step
+                pipe.submit(l, q, k, v, chunk * B_, out_hosts[pipe.i % 2], scores=scores, topc=topc, C=w.topc)
+                st = cache.state(l)
+                e2e_flops += 4.0 * w.head_dim * w.heads * visible_pairs(
+                    w, sum(1 for e in st.kept[:st.n_kept] if e.region != 2))
         chunk += 1
-    e1.record(stream)
+    e1 = pipe.record_done()
     torch.cuda.synchronize()
     e2e_ms, e2e_tot = aggregate_over_ranks(e0.elapsed_time(e1), e2e_flops, dev)
     e2e_value = e2e_tot / (e2e_ms / 1e3) / 1e12
@@ -312,7 +323,8 @@ def run_ours(args, w):
     att_ms = att["ms"] / max(1, att["timed"])
     att_flops_launch = att["flops"] / max(1, att["launches"])
     achieved = att_flops_launch / (att_ms / 1e3) / 1e12
-    traffic = attention_traffic()
+    # the committed capture covers one steady-state layer-pass of the Wan-1.3B stream
+    traffic = attention_traffic() if w.name == "wan13b" else None
     app = prof["append"]
     app_gbs = (app["bytes"] / max(1, app["launches"])) / (app["ms"] / max(1, app["timed"]) / 1e3) / 1e9
 
@@ -341,7 +353,9 @@ def run_ours(args, w):
             "frames_per_s_model": frames / (ms_max / 1e3),
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                    "path": "RollingKVCache.step with pinned host q/k/v/out"},
+                    "path": "RollingKVCache.host_pipeline: pinned host q/k/v in, output back "
+                            "to pinned host, uploads/downloads on their own streams overlapping "
+                            "the kernels (depth 2)"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "kernel": "attention (tcgen05)",
@@ -363,6 +377,69 @@ def run_ours(args, w):
     return 0
 
 
+def run_hbm(args):
+    """HBM-bound kernels at sizes where launch latency does not dominate.
+
+    Three single-layer streams with 40 heads x 128 and 1560-token frames, run
+    through rc_step; the library's per-launch CUDA events isolate the kernel:
+      append    -- fused RoPE + append of a 3-frame chunk (287.5 MB per launch)
+      rotcopy   -- Rolling Sink with static sink semantics: every step rotates
+                   the 15 sink frames again from the raw bank (479 MB)
+      inplace   -- sliding window with an 18-frame sink whose time index moves
+                   by one every step: in-place time rotation (198 MB)
+    Prints one JSON line with GB/s and the fraction of the measured HBM copy
+    bandwidth for each."""
+    import torch
+    from rolling_kv_cache_b200 import binding as B
+    from rolling_kv_cache_b200.cache import RollingKVCache
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    base = rc_synth.WORKLOADS["large"]
+    cases = {
+        "append": (base, "append", None),
+        "rotcopy": (rc_synth.WORKLOADS["rolling_sink"].replace(heads=40, rs_static_semantics=1,
+                                                               dist="normal_frame_mean"), "rerotate", None),
+        "inplace": (base.replace(sink_frames=18, window_frames=3), "rerotate", 1),
+    }
+    res = {}
+    for name, (w, kind, sink_shift) in cases.items():
+        cache = RollingKVCache(make_cfg(w, layers=1), dev)
+        q, k, v = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+                   for x in rc_synth.chunk_qkv(w, 0, 0, 0))
+        out = torch.empty_like(q)
+        chunk = 0
+
+        def step():
+            nonlocal chunk
+            if sink_shift and chunk > 0:
+                cache.reindex(sink_shift, B.RC_REINDEX_SINK)
+            cache.step(0, q, k, v, chunk * w.chunk_frames, out=out)
+            chunk += 1
+
+        for _ in range(w.footprint_frames // w.chunk_frames + 1 + args.warmup):
+            step()
+        torch.cuda.synchronize()
+        B.rc_profile_begin(cache.handle, 8 * args.steps + 16)
+        for _ in range(args.steps):
+            step()
+        torch.cuda.synchronize()
+        prof = B.rc_profile_end(cache.handle)[kind]
+        ms = prof["ms"] / max(1, prof["timed"])
+        by = prof["bytes"] / max(1, prof["launches"])
+        gbs = by / (ms / 1e3) / 1e9
+        res[name] = {"launches": prof["launches"], "ms_per_launch": ms, "bytes_per_launch": by,
+                     "gbs": gbs, "frac": gbs / hbm}
+        cache.close()
+        del q, k, v, out
+    print(json.dumps({"metric": "HBM GB/s of the append and re-rotation kernels", "unit": "GB/s",
+                      "peak": hbm, "peak_source": f"{src} hbm_gbs", "steps": args.steps,
+                      "config": {"heads": 40, "head_dim": 128, "frame_seqlen": 1560}, **res}),
+          flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -374,7 +451,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (small profiling runs)")
+    ap.add_argument("--hbm", action="store_true",
+                    help="measure the HBM-bound append / re-rotation kernels instead")
     args = ap.parse_args()
+    if args.hbm:
+        return run_hbm(args)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     w = rc_synth.WORKLOADS[args.workload]

@@ -112,6 +112,10 @@ class RollingKVCache:
             return out
         return out_dev
 
+    def host_pipeline(self, depth: int = 2) -> "HostPipeline":
+        """Pipelined stepping from host buffers (see HostPipeline)."""
+        return HostPipeline(self, depth)
+
     def _n_frames(self, q, frame_start):
         return self.cfg.chunk_frames if q is None else q.shape[0] // self.cfg.frame_seqlen
 
@@ -166,3 +170,85 @@ class RollingKVCache:
 
     def watchdog_selftest(self, limit_us: int = 20000) -> None:
         B.rc_watchdog_selftest(self.handle, limit_us, self._stream())
+
+
+class HostPipeline:
+    """Steps a cache from host (pinned) q/k/v into host output buffers with
+    the transfers overlapped with the kernels.
+
+    ``depth`` device staging sets are used round robin. Call i's upload runs
+    on a copy-in stream while call i-1 computes on the cache's stream, and
+    call i-1's output download runs on a copy-out stream while call i
+    computes; events order each staging set's reuse. ``submit`` returns at
+    once; ``synchronize`` waits for every download. Host buffers must stay
+    untouched until their call's download is done (after ``synchronize``).
+    """
+
+    def __init__(self, cache: RollingKVCache, depth: int = 2):
+        if cache.device is None:
+            raise RuntimeError("host pipelines need a device cache")
+        self.cache = cache
+        self.depth = max(1, depth)
+        dev = cache.device
+        self.compute = torch.cuda.current_stream(dev)
+        self.copy_in = torch.cuda.Stream(dev)
+        self.copy_out = torch.cuda.Stream(dev)
+        self.sets = []
+        self.i = 0
+
+    def _set(self, q):
+        n = self.i % self.depth
+        if len(self.sets) <= n:
+            dev = self.cache.device
+            self.sets.append(dict(
+                q=torch.empty(q.shape, dtype=torch.bfloat16, device=dev),
+                k=torch.empty(q.shape, dtype=torch.bfloat16, device=dev),
+                v=torch.empty(q.shape, dtype=torch.bfloat16, device=dev),
+                out=torch.empty(q.shape, dtype=torch.bfloat16, device=dev),
+                read=None, downloaded=None))
+        s = self.sets[n]
+        if s["q"].shape != q.shape:
+            raise ValueError("every call of a pipeline must have the same shape")
+        return s
+
+    def submit(self, layer: int, q, k, v, frame_start: int, out_host, lse=None, scores=None,
+               topc=None, C: int = 0) -> None:
+        s = self._set(q)
+        # upload: staging inputs are free once the previous compute using them read them
+        if s["read"] is not None:
+            self.copy_in.wait_event(s["read"])
+        with torch.cuda.stream(self.copy_in):
+            s["q"].copy_(q, non_blocking=True)
+            s["k"].copy_(k, non_blocking=True)
+            s["v"].copy_(v, non_blocking=True)
+            uploaded = torch.cuda.Event()
+            uploaded.record(self.copy_in)
+        # compute: needs the upload, and the staging output downloaded
+        self.compute.wait_event(uploaded)
+        if s["downloaded"] is not None:
+            self.compute.wait_event(s["downloaded"])
+        self.cache.step(layer, s["q"], s["k"], s["v"], frame_start, out=s["out"], lse=lse,
+                        scores=scores, topc=topc, C=C)
+        done = torch.cuda.Event()
+        done.record(self.compute)
+        s["read"] = done
+        # download on its own stream
+        self.copy_out.wait_event(done)
+        with torch.cuda.stream(self.copy_out):
+            out_host.copy_(s["out"], non_blocking=True)
+            dl = torch.cuda.Event()
+            dl.record(self.copy_out)
+        s["downloaded"] = dl
+        self.i += 1
+
+    def record_done(self) -> torch.cuda.Event:
+        """An event on the cache's stream after every submitted download."""
+        for s in self.sets:
+            if s["downloaded"] is not None:
+                self.compute.wait_event(s["downloaded"])
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record(self.compute)
+        return ev
+
+    def synchronize(self) -> None:
+        self.record_done().synchronize()

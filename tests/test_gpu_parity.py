@@ -89,6 +89,28 @@ def test_stream_k_split_units(mask_block):
     r.close()
 
 
+def test_host_pipeline_matches_device_path():
+    # pinned host buffers through the overlapped upload/compute/download
+    # pipeline give the same bytes as device tensors through rc_step
+    w = W["tiny"].replace(heads=4, head_dim=128, grid_h=8, grid_w=16, passes=2, chunks=5)
+    a = RollingKVCache(config_for(w))
+    b = RollingKVCache(config_for(w))
+    pipe = b.host_pipeline(depth=2)
+    outs_a, outs_b = [], []
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        q, k, v = rc_synth.chunk_qkv(w, 0, c, p)
+        outs_a.append(bits_of(a.step(0, dev_bf16(q), dev_bf16(k), dev_bf16(v), g0)))
+        hq, hk, hv = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (q, k, v))
+        ob = torch.empty(hq.shape, dtype=torch.bfloat16, pin_memory=True)
+        pipe.submit(0, hq, hk, hv, g0, ob)
+        outs_b.append(ob)
+    pipe.synchronize()
+    for oa, ob in zip(outs_a, outs_b):
+        assert np.array_equal(oa, ob.view(torch.int16).numpy().view(np.uint16))
+    a.close()
+    b.close()
+
+
 def test_repeat_passes_overwrite():
     w = rc_synth.Workload(name="passes", workload_id=12, layers=2, heads=2, head_dim=128, grid_h=8,
                           grid_w=16, chunk_frames=3, sink_frames=1, window_frames=9,
