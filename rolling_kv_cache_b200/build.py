@@ -35,6 +35,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
            "-o", OUT + ".tmp"]
     if verbose:
         cmd += ["-Xptxas", "-v"]
+    cmd += os.environ.get("RC_NVCC_FLAGS", "").split()  # extra -D tuning flags
     cmd += [os.path.join(CSRC, f) for f in SOURCES]
     cmd += ["-ldl", "-lpthread", "-lrt"]
     r = subprocess.run(cmd, capture_output=True, text=True)

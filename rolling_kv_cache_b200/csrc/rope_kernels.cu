@@ -56,20 +56,20 @@ __device__ __forceinline__ void rot(float& x, float& y, float c, float s) {
   y = ny;
 }
 
+// Thread layout of both kernels: threadIdx.x = 16-byte chunk of a head row
+// (d/8 lanes cover one row), threadIdx.y = row within the block; rows are
+// walked grid-stride in 32-bit arithmetic.
 __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ AppendParams p) {
-  const int chunks = p.d >> 3;
-  const long long total = (long long)p.n_tok * p.H * chunks;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int c8 = (int)(i % chunks);
-    const long long th = i / chunks;
-    const int h = (int)(th % p.H);
-    const int tok = (int)(th / p.H);
+  const int c8 = threadIdx.x;
+  const int rows = p.n_tok * p.H;  // (token, head) rows in input order
+  for (int row = blockIdx.x * blockDim.y + threadIdx.y; row < rows; row += gridDim.x * blockDim.y) {
+    const int tok = row / p.H;
+    const int h = row - tok * p.H;
     const int r = tok / p.F;
     const int n_in = tok - r * p.F;
     const int hr = n_in / p.rt.grid_w;
     const int wc = n_in - hr * p.rt.grid_w;
-    const size_t src = ((size_t)tok * p.H + h) * p.d + c8 * 8;
+    const size_t src = (size_t)row * p.d + c8 * 8;
     uint4 uq = __ldg(reinterpret_cast<const uint4*>(p.q + src));
     uint4 uk = __ldg(reinterpret_cast<const uint4*>(p.k + src));
     uint4 uv = __ldg(reinterpret_cast<const uint4*>(p.v + src));
@@ -97,26 +97,29 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
   }
 }
 
-// One job per blockIdx.y. Rotate-copy rewrites the whole key row from the
-// pristine raw source at the job's target time (and copies V when the slot's
-// content changes); in-place composes R_t(delta) onto the stored key, touching
-// only the chunks that hold time pairs.
+// One job per blockIdx.y; rows ordered (head, token in frame) so a warp
+// writes whole consecutive rows of one head's slot. Rotate-copy rewrites the
+// key row from the pristine raw source at the job's target time (and copies
+// V when the slot's content changes); in-place composes R_t(delta) onto the
+// stored key and touches only the chunks that hold time pairs.
 __global__ void __launch_bounds__(256) rerotate_kernel(const __grid_constant__ RerotateParams p) {
   const RerotateJob& jb = p.job[blockIdx.y];
-  const bool inplace = jb.mode == 1;
-  const int chunks = inplace ? (2 * p.rt.pt + 7) / 8 : p.d / 8;
-  const long long total = (long long)p.F * p.H * chunks;
-  const float sgn = jb.delta < 0 ? -1.f : 1.f;
-  const int adelta = jb.delta < 0 ? -jb.delta : jb.delta;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int c8 = (int)(i % chunks);
-    const long long th = i / chunks;
-    const int h = (int)(th % p.H);
-    const int n_in = (int)(th / p.H);
-    const size_t dst = ((size_t)h * p.cap + (size_t)jb.dst_slot * p.F + n_in) * p.d + c8 * 8;
-    float f[8];
-    if (inplace) {
+  const int rows = p.F * p.H;
+  if (jb.mode == 1) {
+    // in place: only the ct chunks holding time pairs; the block's threads
+    // are packed densely over (row, chunk) so every lane has work
+    const int ct = (2 * p.rt.pt + 7) / 8;
+    const float sgn = jb.delta < 0 ? -1.f : 1.f;
+    const int adelta = jb.delta < 0 ? -jb.delta : jb.delta;
+    const int nthr = blockDim.x * blockDim.y;
+    const int total = rows * ct;
+    for (int i = blockIdx.x * nthr + threadIdx.y * blockDim.x + threadIdx.x; i < total; i += gridDim.x * nthr) {
+      const int row = i / ct;
+      const int c8 = i - row * ct;
+      const int h = row / p.F;
+      const int n_in = row - h * p.F;
+      const size_t dst = ((size_t)h * p.cap + (size_t)jb.dst_slot * p.F + n_in) * p.d + c8 * 8;
+      float f[8];
       uint4 u = *reinterpret_cast<const uint4*>(p.kc + dst);
       unpack8(u, f);
 #pragma unroll
@@ -128,7 +131,16 @@ __global__ void __launch_bounds__(256) rerotate_kernel(const __grid_constant__ R
         }
       }
       *reinterpret_cast<uint4*>(p.kc + dst) = pack8(f);
-    } else {
+    }
+    return;
+  }
+  const int c8 = threadIdx.x;
+  for (int row = blockIdx.x * blockDim.y + threadIdx.y; row < rows; row += gridDim.x * blockDim.y) {
+    const int h = row / p.F;
+    const int n_in = row - h * p.F;
+    const size_t dst = ((size_t)h * p.cap + (size_t)jb.dst_slot * p.F + n_in) * p.d + c8 * 8;
+    float f[8];
+    {
       const int hr = n_in / p.rt.grid_w;
       const int wc = n_in - hr * p.rt.grid_w;
       const size_t src = ((size_t)h * p.raw_cap + (size_t)jb.src_frame * p.F + n_in) * p.d + c8 * 8;
@@ -160,23 +172,25 @@ int sm_count() {
 }  // namespace
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
-  const long long total = (long long)p.n_tok * p.H * (p.d / 8);
-  if (total == 0) return cudaSuccess;
-  long long blocks = (total + 255) / 256;
-  const long long cap = (long long)sm_count() * 8;  // 8 resident 256-thread blocks per SM
+  const int rows = p.n_tok * p.H;
+  if (rows == 0) return cudaSuccess;
+  const dim3 block(p.d / 8, 256 / (p.d / 8));
+  int blocks = (rows + block.y - 1) / block.y;
+  const int cap = sm_count() * 8;  // 8 resident 256-thread blocks per SM
   if (blocks > cap) blocks = cap;
-  append_kernel<<<(unsigned)blocks, 256, 0, s>>>(p);
+  append_kernel<<<blocks, block, 0, s>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_rerotate(const RerotateParams& p, cudaStream_t s) {
   if (p.n_jobs == 0) return cudaSuccess;
-  const long long per_job = (long long)p.F * p.H * (p.d / 8);
-  long long bx = (per_job + 255) / 256;
-  const long long cap = ((long long)sm_count() * 8 + p.n_jobs - 1) / p.n_jobs;
+  const dim3 block(p.d / 8, 256 / (p.d / 8));
+  const int rows = p.F * p.H;
+  int bx = (rows + block.y - 1) / block.y;
+  const int cap = (sm_count() * 8 + p.n_jobs - 1) / p.n_jobs;
   if (bx > cap) bx = cap;
   if (bx < 1) bx = 1;
-  rerotate_kernel<<<dim3((unsigned)bx, (unsigned)p.n_jobs), 256, 0, s>>>(p);
+  rerotate_kernel<<<dim3(bx, p.n_jobs), block, 0, s>>>(p);
   return cudaGetLastError();
 }
 
