@@ -327,19 +327,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         ptx::tc_fence_after();
         // columns [0, lim) of this row are visible (the whole row or a ragged tail is masked)
         const int lim = (t.rank < 0 || t.rank <= my_rank) ? t.nvalid : 0;
-        // pass 1: row maximum of the raw scores
+        // pass 1: row maximum of the raw scores (two 32-column loads in flight per wait)
         float mx = -INFINITY;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t r[32];
-          ptx::tmem_ld32(tS + cc * 32, r);
+        for (int cc = 0; cc < 4; cc += 2) {
+          uint32_t ra[32], rb[32];
+          ptx::tmem_ld32(tS + cc * 32, ra);
+          ptx::tmem_ld32(tS + (cc + 1) * 32, rb);
           ptx::tmem_ld_wait();
           if (lim == kTileRows) {
 #pragma unroll
-            for (int k = 0; k < 32; ++k) mx = fmaxf(mx, __uint_as_float(r[k]));
+            for (int k = 0; k < 32; ++k) mx = fmaxf(mx, fmaxf(__uint_as_float(ra[k]), __uint_as_float(rb[k])));
           } else {
 #pragma unroll
-            for (int k = 0; k < 32; ++k) mx = fmaxf(mx, cc * 32 + k < lim ? __uint_as_float(r[k]) : -INFINITY);
+            for (int k = 0; k < 32; ++k) {
+              mx = fmaxf(mx, cc * 32 + k < lim ? __uint_as_float(ra[k]) : -INFINITY);
+              mx = fmaxf(mx, (cc + 1) * 32 + k < lim ? __uint_as_float(rb[k]) : -INFINITY);
+            }
           }
         }
         const float m_new = fmaxf(m, mx);
@@ -367,11 +371,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         // 64 columns; chunk cc's P columns [16cc, 16cc+16) lie in S columns
         // already read, so the overwrite never races a later read.
         float sum = 0.f;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t r[32];
-          ptx::tmem_ld32(tS + cc * 32, r);
-          ptx::tmem_ld_wait();
+        auto emit = [&](const uint32_t (&r)[32], int cc) {
           uint32_t pk[16];
           if (lim == kTileRows) {
 #pragma unroll
@@ -392,6 +392,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
             }
           }
           ptx::tmem_st16(tS + cc * 16, pk);
+        };
+#pragma unroll
+        for (int cc = 0; cc < 4; cc += 2) {
+          uint32_t ra[32], rb[32];
+          ptx::tmem_ld32(tS + cc * 32, ra);
+          ptx::tmem_ld32(tS + (cc + 1) * 32, rb);
+          ptx::tmem_ld_wait();
+          emit(ra, cc);
+          emit(rb, cc + 1);
         }
         ptx::tmem_st_wait();
         l += sum;
