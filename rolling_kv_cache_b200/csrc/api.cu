@@ -490,6 +490,13 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
     sp.Nq = Nq;
     sp.H = H;
     sp.scale_log2 = at.scale_log2;
+    sp.n_pairs = (Nq + 255) / 256;
+    sp.tiles = 0;
+    for (int i = 0; i < sp.n_segs; ++i) sp.tiles += (sp.seg[i].len + 127) / 128;
+    {
+      const long long work = (long long)H * sp.n_pairs * sp.tiles;
+      sp.n_ctas = (int)std::min<long long>(c->sm_count, work);
+    }
     {
       Timed tm(c->prof, RC_KERNEL_SCORES, s, 2.0 * d * H * Nq * (double)plan.cand.size() * F, 0.0);
       if (cudaError_t e = rc::launch_scores(sp, d, s)) return cuda_err(e, "scores launch");

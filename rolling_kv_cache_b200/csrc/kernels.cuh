@@ -103,6 +103,9 @@ struct alignas(64) ScoreParams {
   float scale_log2;
   int n_segs;
   KvSegment seg[kMaxSegs];
+  int n_pairs;   // 256-query pairs per head
+  int tiles;     // candidate KV tiles (every pair walks all of them)
+  int n_ctas;    // persistent grid
 };
 
 // K6b: gather scores to logical order + top-C.

@@ -5,66 +5,117 @@
 // over heads and queries of the softmax probability the attention used,
 // p = exp(q.k_j / sqrt(d) - LSE), with the attention's final LSE. This is a
 // second Q K^T pass over the history tiles only (sink and current chunk are
-// not candidates).
+// not candidates, and every query sees every candidate).
 //
-// One CTA = one 128-query tile of one head; warp 0 loads Q and K tiles
-// (TMA, 2-stage ring), warp 1 issues S = Q K^T into TMEM, warps 4..7 turn a
-// row of S into probabilities and reduce columns. Bounded waits, no trap.
+// Persistent CTAs walk (head, query pair, KV tile) items in equal contiguous
+// ranges; column sums go to global memory with atomics, so a pair cut
+// between CTAs needs no merge. Per CTA, two 128-query tiles share each K tile:
+//   warps 0-3 / 4-7  softmax of Q0 / Q1: P = 2^(s c - lse2) as bf16 into
+//                    shared memory ([query][key], 128-byte swizzle)
+//   warp 8           TMA producer (Q pair per job, K tiles in a 2-stage ring)
+//   warps 9 / 10     one MMA issuer per query tile (warp 9 also owns TMEM)
+// The column sum itself runs on the tensor core: D'_g = P_g^T 1 with P_g^T
+// read MN-major from shared memory (M = 128 keys, N = 16, K = 128 queries);
+// lane j of D'_g holds key j's sum over the tile's queries, which group g
+// reads one tile later and adds to the score buffer.
+// TMEM: S0 [0,128), S1 [128,256), D'_0 [256,288), D'_1 [288,320) (2 buffers each).
+// Bounded waits (RC_ETIMEOUT in the status word), no trap.
 #include "attn_common.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
-
-#include <cuda_bf16.h>
 
 namespace rc {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kSoftmaxWarp0 = 4;
-constexpr int kStatusTimeout = RC_ETIMEOUT;
+constexpr int kScoreThreads = 384;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kPTileBytes = 128 * 128 * 2;  // P: 128 queries x 128 keys bf16
+constexpr uint32_t kOnesBytes = 16 * 128 * 2;    // B = ones: 16 x 128 bf16
 
 template <int D>
-struct Layout {
+struct ScoreLayout {
   static constexpr int kSub = D / 64;
-  static constexpr uint32_t kTile = kSubTileBytes * kSub;
-  static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kK = kQ + kTile;           // 2 stages
-  static constexpr uint32_t kV = kK + 2 * kTile;       // 2 stages
-  static constexpr uint32_t kBytes = kV + 2 * kTile;
-  static constexpr uint32_t kDynSmem = kBytes + 1024;  // alignment slack
+  static constexpr uint32_t kTile = kSubTileBytes * kSub;  // Q or K tile: 128 rows x D
+  static constexpr uint32_t kQ = 0;                         // Q0, Q1
+  static constexpr uint32_t kK = 2 * kTile;                 // 2 stages
+  static constexpr uint32_t kP = 4 * kTile;                 // P0, P1
+  static constexpr uint32_t kOnes = kP + 2 * kPTileBytes;
+  static constexpr uint32_t kBytes = kOnes + kOnesBytes;
+  static constexpr uint32_t kDynSmem = kBytes + 1024;
+};
+
+struct ScoreJob {
+  int h, q0, kv_lo, kv_hi;
+  bool has1;
+};
+
+// Equal contiguous ranges of the W = H * NP * T work items (head, pair, tile).
+struct ScoreScheduler {
+  const ScoreParams* p;
+  long long pos, end;
+  __device__ void init(const ScoreParams& prm) {
+    p = &prm;
+    const long long W = (long long)prm.H * prm.n_pairs * prm.tiles;
+    pos = (long long)blockIdx.x * W / gridDim.x;
+    end = (long long)(blockIdx.x + 1) * W / gridDim.x;
+  }
+  __device__ bool next(ScoreJob& j) {
+    if (pos >= end) return false;
+    const long long unit = pos / p->tiles;
+    const int off = (int)(pos - unit * p->tiles);
+    const int len = (int)min((long long)(p->tiles - off), end - pos);
+    pos += len;
+    j.h = (int)(unit / p->n_pairs);
+    j.q0 = (int)(unit % p->n_pairs) * 2 * kTileRows;
+    j.kv_lo = off;
+    j.kv_hi = off + len;
+    // both tiles always: rows past Nq load as zeros and get lse2 = +inf, so
+    // their P is exactly 0 (keeps the two issuers' barrier phases in step)
+    j.has1 = true;
+    return true;
+  }
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) score_kernel(const __grid_constant__ ScoreParams p) {
-  using L = Layout<D>;
+__global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const __grid_constant__ ScoreParams p) {
+  using L = ScoreLayout<D>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_q, bar_k[2], bar_kv_free[2], bar_s, bar_sfree, bar_fin;
+  __shared__ uint64_t bar_q, bar_qe, bar_kf[2], bar_ke[2], bar_s[2], bar_sfree[2], bar_p[2], bar_pfree[2],
+      bar_dfull[2][2], bar_dfree[2][2], bar_fin[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
-  __shared__ float red[4][128];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, h = blockIdx.y;
   const uint32_t base_u32 = (ptx::smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_u32 - ptx::smem_u32(smem_raw));
-  const int q0 = qt * kTileRows;
-  const int T = count_tiles(p.seg, p.n_segs, 0x7fffffff);
 
+  // B operand of the column sum: all ones (layout-free)
+  for (uint32_t i = threadIdx.x; i < kOnesBytes / 4; i += blockDim.x)
+    reinterpret_cast<uint32_t*>(base + L::kOnes)[i] = 0x3F803F80u;
+  ptx::fence_proxy_async_smem();
   if (threadIdx.x == 0) {
     ptx::mbar_init(&bar_q, 1);
+    ptx::mbar_init(&bar_qe, 2);
     for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(&bar_k[i], 1);
-      ptx::mbar_init(&bar_kv_free[i], 1);
+      ptx::mbar_init(&bar_kf[i], 1);
+      ptx::mbar_init(&bar_ke[i], 2);
+      ptx::mbar_init(&bar_s[i], 1);
+      ptx::mbar_init(&bar_sfree[i], 128);
+      ptx::mbar_init(&bar_p[i], 128);
+      ptx::mbar_init(&bar_pfree[i], 1);
+      for (int b = 0; b < 2; ++b) {
+        ptx::mbar_init(&bar_dfull[i][b], 1);
+        ptx::mbar_init(&bar_dfree[i][b], 128);
+      }
+      ptx::mbar_init(&bar_fin[i], 1);
     }
-    ptx::mbar_init(&bar_s, 1);
-    ptx::mbar_init(&bar_sfree, 128);
-    ptx::mbar_init(&bar_fin, 1);
     abort_sh = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 1) {
-    ptx::tmem_alloc(&tmem_base_sh, 128);
+  if (warp == kMmaWarp) {
+    ptx::tmem_alloc(&tmem_base_sh, 512);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -72,109 +123,201 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(const __grid_constan
   ptx::tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
   volatile int* abort = &abort_sh;
+  int dummy_abort = 0;
+  volatile int* noabort = reinterpret_cast<volatile int*>(&dummy_abort);
+  ScoreScheduler sc;
+  sc.init(p);
+  ScoreJob jb;
 
-  if (warp == 0 && lane == 0) {
-    ptx::mbar_arrive_expect_tx(&bar_q, L::kTile);
-    for (int j = 0; j < L::kSub; ++j)
-      ptx::tma_load_3d(&p.tm_q, &bar_q, base + L::kQ + j * kSubTileBytes, 64 * j, q0, h);
-    TileWalker wk{p.seg, p.n_segs, 0x7fffffff};
-    Tile t;
-    int issued[2] = {0, 0};
-    for (int i = 0; wk.next(t); ++i) {
-      const int st = i & 1;
-      if (i >= 2 && !ptx::mbar_wait(&bar_kv_free[st], ((i >> 1) - 1) & 1, abort, p.status, kStatusTimeout))
-        break;
-      ptx::mbar_arrive_expect_tx(&bar_k[st], L::kTile);
-      for (int j = 0; j < L::kSub; ++j)
-        ptx::tma_load_3d(&p.tm_k, &bar_k[st], base + L::kK + st * L::kTile + j * kSubTileBytes, 64 * j,
-                         t.tok, h);
-      issued[st]++;
+  if (warp == kProducerWarp && lane == 0) {
+    // ---------------------------------------------------------- producer
+    int nq = 0, g = 0, nk[2] = {0, 0};
+    bool ok = true;
+    while (ok && sc.next(jb)) {
+      if (nq > 0 && !ptx::mbar_wait(&bar_qe, (nq - 1) & 1, abort, p.status, RC_ETIMEOUT)) break;
+      ptx::mbar_arrive_expect_tx(&bar_q, (jb.has1 ? 2 : 1) * L::kTile);
+      for (int i = 0; i < (jb.has1 ? 2 : 1); ++i)
+        for (int k = 0; k < L::kSub; ++k)
+          ptx::tma_load_3d(&p.tm_q, &bar_q, base + L::kQ + i * L::kTile + k * kSubTileBytes, 64 * k,
+                           jb.q0 + i * kTileRows, jb.h);
+      ++nq;
+      TileWalker wk{p.seg, p.n_segs, 0x7fffffff};
+      wk.seek(jb.kv_lo);
+      Tile t;
+      for (int j = jb.kv_lo; j < jb.kv_hi && wk.next(t); ++j, ++g) {
+        const int st = g & 1;
+        if (g >= 2 && !ptx::mbar_wait(&bar_ke[st], ((g >> 1) - 1) & 1, abort, p.status, RC_ETIMEOUT)) {
+          ok = false;
+          break;
+        }
+        ptx::mbar_arrive_expect_tx(&bar_kf[st], L::kTile);
+        for (int k = 0; k < L::kSub; ++k)
+          ptx::tma_load_3d(&p.tm_k, &bar_kf[st], base + L::kK + st * L::kTile + k * kSubTileBytes, 64 * k, t.tok,
+                           jb.h);
+        nk[st]++;
+      }
     }
-    int dummy = 0;
-    volatile int* noabort = reinterpret_cast<volatile int*>(&dummy);
-    ptx::mbar_wait(&bar_q, 0, noabort, p.status, kStatusTimeout);
+    if (nq) ptx::mbar_wait(&bar_q, (nq - 1) & 1, noabort, p.status, RC_ETIMEOUT);
     for (int st = 0; st < 2; ++st)
-      if (issued[st]) ptx::mbar_wait(&bar_k[st], (issued[st] - 1) & 1, noabort, p.status, kStatusTimeout);
-  } else if (warp == 1 && lane == 0) {
+      if (nk[st]) ptx::mbar_wait(&bar_kf[st], (nk[st] - 1) & 1, noabort, p.status, RC_ETIMEOUT);
+  } else if ((warp == kMmaWarp || warp == kMmaWarp + 1) && lane == 0) {
+    // ---------------------------------------------------------- MMA issuers
+    // one thread per query tile, so the two groups' pipelines never wait on
+    // each other; K stages and the Q pair are released by both (count 2)
+    const int g = warp - kMmaWarp;
     constexpr uint32_t idesc_s = ptx::idesc_bf16(128, 128, 0, 0);
-    const uint32_t sQ = base_u32 + L::kQ;
-    bool ok = ptx::mbar_wait(&bar_q, 0, abort, p.status, kStatusTimeout);
-    for (int i = 0; ok && i < T; ++i) {
-      const int st = i & 1;
+    constexpr uint32_t idesc_c = ptx::idesc_bf16(128, 16, 1, 0);  // A = P^T (MN-major), B = ones (K-major)
+    const uint32_t sQg = base_u32 + L::kQ + g * L::kTile;
+    const uint32_t sP = base_u32 + L::kP + g * kPTileBytes;
+    const uint32_t sOnes = base_u32 + L::kOnes;
+    auto issue_s = [&](int st) {
       const uint32_t sK = base_u32 + L::kK + st * L::kTile;
-      if (!ptx::mbar_wait(&bar_k[st], (i >> 1) & 1, abort, p.status, kStatusTimeout)) break;
-      if (i > 0 && !ptx::mbar_wait(&bar_sfree, (i - 1) & 1, abort, p.status, kStatusTimeout)) break;
-      ptx::tc_fence_after();
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
         const uint32_t off = (ks >> 2) * kSubTileBytes + (ks & 3) * 32;
-        ptx::mma_ss(tmem, ptx::sdesc_sw128(sQ + off, 16, 1024), ptx::sdesc_sw128(sK + off, 16, 1024), idesc_s,
-                    ks > 0);
+        ptx::mma_ss(tmem + g * 128, ptx::sdesc_sw128(sQg + off, 16, 1024), ptx::sdesc_sw128(sK + off, 16, 1024),
+                    idesc_s, ks > 0);
       }
-      ptx::mma_commit(&bar_s);
-      ptx::mma_commit(&bar_kv_free[st]);
+      ptx::mma_commit(&bar_s[g]);
+    };
+    int nq = 0, gk = 0, gt = 0, gd = 0;
+    bool ok = true;
+    while (ok && sc.next(jb)) {
+      const int n = jb.kv_hi - jb.kv_lo;
+      if (!ptx::mbar_wait(&bar_q, nq & 1, abort, p.status, RC_ETIMEOUT)) break;
+      ++nq;
+      if (!ptx::mbar_wait(&bar_kf[gk & 1], (gk >> 1) & 1, abort, p.status, RC_ETIMEOUT)) break;
+      if (gt > 0 && !ptx::mbar_wait(&bar_sfree[g], (gt - 1) & 1, abort, p.status, RC_ETIMEOUT)) break;
+      ptx::tc_fence_after();
+      issue_s(gk & 1);
+      ptx::mma_commit(&bar_ke[gk & 1]);
+      if (n == 1) ptx::mma_commit(&bar_qe);
+      for (int j = 0; j < n; ++j, ++gk, ++gt, ++gd) {
+        if (j + 1 < n) {  // S of the next tile once this one's S has been read
+          const int st1 = (gk + 1) & 1;
+          if (!ptx::mbar_wait(&bar_kf[st1], ((gk + 1) >> 1) & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
+          if (!ptx::mbar_wait(&bar_sfree[g], gt & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
+          ptx::tc_fence_after();
+          issue_s(st1);
+          ptx::mma_commit(&bar_ke[st1]);
+          if (j + 2 == n) ptx::mma_commit(&bar_qe);
+        }
+        const int db = gd & 1;
+        if (gd >= 2 && !ptx::mbar_wait(&bar_dfree[g][db], ((gd >> 1) - 1) & 1, abort, p.status, RC_ETIMEOUT)) {
+          ok = false;
+          break;
+        }
+        if (!ptx::mbar_wait(&bar_p[g], gt & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < kTileRows / 16; ++ks)
+          ptx::mma_ss(tmem + 256 + g * 32 + db * 16, ptx::sdesc_sw128(sP + ks * 2048, kSubTileBytes, 1024),
+                      ptx::sdesc_sw128(sOnes + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024), idesc_c, ks > 0);
+        ptx::mma_commit(&bar_pfree[g]);
+        ptx::mma_commit(&bar_dfull[g][db]);
+      }
     }
-    int dummy = 0;
-    ptx::mma_commit(&bar_fin);
-    ptx::mbar_wait(&bar_fin, 0, reinterpret_cast<volatile int*>(&dummy), p.status, kStatusTimeout);
-  } else if (warp >= kSoftmaxWarp0) {
+    ptx::mma_commit(&bar_fin[g]);
+    ptx::mbar_wait(&bar_fin[g], 0, noabort, p.status, RC_ETIMEOUT);
+  } else if (warp < 8) {
+    // ---------------------------------------------------------- softmax
+    const int grp = warp >> 2;
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
-    const int qtok = q0 + row;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const float lse2 = qtok < p.Nq ? p.lse[(size_t)h * p.Nq + qtok] * 1.4426950408889634f : INFINITY;
-    TileWalker wk{p.seg, p.n_segs, 0x7fffffff};
-    Tile t;
-    for (int i = 0; wk.next(t); ++i) {
-      if (!ptx::mbar_wait(&bar_s, i & 1, abort, p.status, kStatusTimeout)) break;
+    const uint32_t tS = tmem + lane_off + grp * 128;
+    uint8_t* sP = base + L::kP + grp * kPTileBytes;
+    const float c = p.scale_log2;
+    int gs = 0;            // this group's tiles (phases of s / sfree / p / pfree)
+    int gd = 0;            // D' sums read by this group
+    int prev_tok = 0, prev_nvalid = 0;
+    bool have_prev = false;
+    // add the previous tile's key sums (lane j of this group's D' = key j) to the scores
+    auto drain = [&]() -> bool {
+      if (!have_prev) return true;
+      const int db = gd & 1;
+      if (!ptx::mbar_wait(&bar_dfull[grp][db], (gd >> 1) & 1, abort, p.status, RC_ETIMEOUT)) return false;
       ptx::tc_fence_after();
-      float colsum[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t s[32];
-        ptx::tmem_ld32(tmem + lane_off + c * 32, s);
-        ptx::tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) colsum[c * 32 + j] = ptx::ex2(__uint_as_float(s[j]) * p.scale_log2 - lse2);
-      }
+      uint32_t r[32];
+      ptx::tmem_ld32(tmem + lane_off + 256 + grp * 32 + db * 16, r);
+      ptx::tmem_ld_wait();
+      if (row < prev_nvalid) atomicAdd(p.score_phys + prev_tok + row, __uint_as_float(r[0]));
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&bar_sfree);
-      // transpose-reduce over the warp's 32 rows: afterwards lane l holds
-      // the 32-row sum of column (c*32 + l) in colsum[c*32]
+      ptx::mbar_arrive(&bar_dfree[grp][db]);
+      ++gd;
+      have_prev = false;
+      return true;
+    };
+    bool ok = true;
+    while (ok && sc.next(jb)) {
+      if (*abort) break;
+      const int qtok = jb.q0 + grp * kTileRows + row;
+      const float lse2 = qtok < p.Nq ? p.lse[(size_t)jb.h * p.Nq + qtok] * 1.4426950408889634f : INFINITY;
+      TileWalker wk{p.seg, p.n_segs, 0x7fffffff};
+      wk.seek(jb.kv_lo);
+      Tile t;
+      for (int j = jb.kv_lo; j < jb.kv_hi && wk.next(t); ++j) {
+        if (!ptx::mbar_wait(&bar_s[grp], gs & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
+        ptx::tc_fence_after();
+        // P smem of the previous tile must have been read by its column-sum MMA
+        if (gs > 0 && !ptx::mbar_wait(&bar_pfree[grp], (gs - 1) & 1, abort, p.status, RC_ETIMEOUT)) {
+          ok = false;
+          break;
+        }
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float* v = colsum + c * 32;
+        for (int half = 0; half < 2; ++half) {
+          uint32_t ra[32], rb[32];
+          ptx::tmem_ld32(tS + half * 64, ra);
+          ptx::tmem_ld32(tS + half * 64 + 32, rb);
+          ptx::tmem_ld_wait();
+          if (half == 1) {  // S fully read: the MMA may overwrite it
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&bar_sfree[grp]);
+          }
+          uint32_t pk[32];
 #pragma unroll
-        for (int k = 16; k >= 1; k >>= 1) {
-          const bool upper = (lane & k) != 0;
+          for (int k = 0; k < 16; ++k) {
+            const int col = half * 64 + 2 * k;
+            const float a = col < t.nvalid ? ptx::ex2(fmaf(__uint_as_float(ra[2 * k]), c, -lse2)) : 0.f;
+            const float b = col + 1 < t.nvalid ? ptx::ex2(fmaf(__uint_as_float(ra[2 * k + 1]), c, -lse2)) : 0.f;
+            pk[k] = ptx::pack_bf16x2(a, b);
+          }
 #pragma unroll
-          for (int j = 0; j < k; ++j) {
-            const float send = upper ? v[j] : v[j + k];
-            const float keep = upper ? v[j + k] : v[j];
-            v[j] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+          for (int k = 0; k < 16; ++k) {
+            const int col = half * 64 + 32 + 2 * k;
+            const float a = col < t.nvalid ? ptx::ex2(fmaf(__uint_as_float(rb[2 * k]), c, -lse2)) : 0.f;
+            const float b = col + 1 < t.nvalid ? ptx::ex2(fmaf(__uint_as_float(rb[2 * k + 1]), c, -lse2)) : 0.f;
+            pk[16 + k] = ptx::pack_bf16x2(a, b);
+          }
+          // P[row][64 half .. 64 half + 63] -> sub-tile `half`, 8 chunks of 16 bytes, swizzled
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+            *reinterpret_cast<uint4*>(sP + half * kSubTileBytes + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
           }
         }
-        red[wq][c * 32 + lane] = v[0];
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(&bar_p[grp]);
+        ++gs;
+        if (!drain()) { ok = false; break; }
+        prev_tok = t.tok;
+        prev_nvalid = t.nvalid;
+        have_prev = true;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      {
-        const float tot = red[0][row] + red[1][row] + red[2][row] + red[3][row];
-        if (row < t.nvalid) atomicAdd(p.score_phys + t.tok + row, tot);
-      }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
     }
+    if (ok) drain();
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, 128);
+    ptx::tmem_dealloc(tmem, 512);
   }
 }
 
 template <int D>
 cudaError_t launch_scores_d(const ScoreParams& p, cudaStream_t s) {
-  using L = Layout<D>;
+  using L = ScoreLayout<D>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -182,15 +325,14 @@ cudaError_t launch_scores_d(const ScoreParams& p, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid((p.Nq + kTileRows - 1) / kTileRows, p.H);
-  score_kernel<D><<<grid, kThreads, L::kDynSmem, s>>>(p);
+  score_kernel<D><<<p.n_ctas, kScoreThreads, L::kDynSmem, s>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_scores(const ScoreParams& p, int head_dim, cudaStream_t s) {
-  if (p.Nq <= 0 || p.n_segs == 0) return cudaSuccess;
+  if (p.Nq <= 0 || p.n_segs == 0 || p.tiles == 0 || p.n_ctas <= 0) return cudaSuccess;
   return head_dim == 64 ? launch_scores_d<64>(p, s) : launch_scores_d<128>(p, s);
 }
 
