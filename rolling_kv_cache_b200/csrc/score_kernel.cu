@@ -10,14 +10,17 @@
 // Persistent CTAs walk (head, query pair, KV tile) items in equal contiguous
 // ranges; column sums go to global memory with atomics, so a pair cut
 // between CTAs needs no merge. Per CTA, two 128-query tiles share each K tile:
-//   warps 0-3 / 4-7  softmax of Q0 / Q1: P = 2^(s c - lse2) as bf16 into
-//                    shared memory ([query][key], 128-byte swizzle)
-//   warp 8           TMA producer (Q pair per job, K tiles in a 2-stage ring)
-//   warps 9 / 10     one MMA issuer per query tile (warp 9 also owns TMEM)
+//   warps 0-7 / 8-15  softmax of Q0 / Q1: P = 2^(s c - lse2) as bf16 into
+//                     shared memory ([query][key], 128-byte swizzle); each
+//                     warp takes 32 rows x 64 keys, so four softmax warps
+//                     share each SM sub-partition's exp2 unit
+//   warp 16           TMA producer (Q pair per job, K tiles in a 2-stage ring)
+//   warps 17 / 18     one MMA issuer per query tile (warp 17 also owns TMEM)
 // The column sum itself runs on the tensor core: D'_g = P_g^T 1 with P_g^T
 // read MN-major from shared memory (M = 128 keys, N = 16, K = 128 queries);
 // lane j of D'_g holds key j's sum over the tile's queries, which group g
-// reads one tile later and adds to the score buffer.
+// reads one tile later (its two column halves in turn) and adds to the score
+// buffer.
 // TMEM: S0 [0,128), S1 [128,256), D'_0 [256,288), D'_1 [288,320) (2 buffers each).
 // Bounded waits (RC_ETIMEOUT in the status word), no trap.
 #include "attn_common.cuh"
@@ -28,9 +31,10 @@ namespace rc {
 
 namespace {
 
-constexpr int kScoreThreads = 384;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kSoftmaxWarps = 16;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;  // and 18
+constexpr int kScoreThreads = 19 * 32;
 constexpr uint32_t kPTileBytes = 128 * 128 * 2;  // P: 128 queries x 128 keys bf16
 constexpr uint32_t kOnesBytes = 16 * 128 * 2;    // B = ones: 16 x 128 bf16
 
@@ -78,6 +82,29 @@ struct ScoreScheduler {
   }
 };
 
+// P = 2^(s c - lse2) of 32 keys of one row (S columns c0 .. c0 + 31 of this
+// warp's half) as bf16, into the row's four 16-byte chunks c0/8 .. c0/8 + 3 of
+// the 128-byte-swizzled sub-tile. Keys at or past lim (ragged tile end) get 0.
+template <bool kCheck>
+__device__ __forceinline__ void exp_store(const uint32_t (&r)[32], int c0, int lim, float c, float lse2,
+                                          uint8_t* sProw, int row) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    float a = ptx::ex2(fmaf(__uint_as_float(r[2 * k]), c, -lse2));
+    float b = ptx::ex2(fmaf(__uint_as_float(r[2 * k + 1]), c, -lse2));
+    if (kCheck) {
+      if (c0 + 2 * k >= lim) a = 0.f;
+      if (c0 + 2 * k + 1 >= lim) b = 0.f;
+    }
+    pk[k] = ptx::pack_bf16x2(a, b);
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<uint4*>(sProw + (((c0 / 8 + q) ^ (row & 7)) << 4)) =
+        make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const __grid_constant__ ScoreParams p) {
   using L = ScoreLayout<D>;
@@ -102,8 +129,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const __grid_co
       ptx::mbar_init(&bar_kf[i], 1);
       ptx::mbar_init(&bar_ke[i], 2);
       ptx::mbar_init(&bar_s[i], 1);
-      ptx::mbar_init(&bar_sfree[i], 128);
-      ptx::mbar_init(&bar_p[i], 128);
+      ptx::mbar_init(&bar_sfree[i], 256);
+      ptx::mbar_init(&bar_p[i], 256);
       ptx::mbar_init(&bar_pfree[i], 1);
       for (int b = 0; b < 2; ++b) {
         ptx::mbar_init(&bar_dfull[i][b], 1);
@@ -219,33 +246,37 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const __grid_co
     }
     ptx::mma_commit(&bar_fin[g]);
     ptx::mbar_wait(&bar_fin[g], 0, noabort, p.status, RC_ETIMEOUT);
-  } else if (warp < 8) {
+  } else if (warp < kSoftmaxWarps) {
     // ---------------------------------------------------------- softmax
-    const int grp = warp >> 2;
+    // group g = warp / 8 owns query tile g; within it warp w reads TMEM lane
+    // quarter w % 4 (rows) and column half (w / 4) % 2 (keys [64 ch, 64 ch + 64))
+    const int grp = warp >> 3;
+    const int ch = (warp >> 2) & 1;
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + grp * 128;
-    uint8_t* sP = base + L::kP + grp * kPTileBytes;
+    const uint32_t tS = tmem + lane_off + grp * 128 + ch * 64;
+    uint8_t* sProw = base + L::kP + grp * kPTileBytes + ch * kSubTileBytes + row * 128;
     const float c = p.scale_log2;
     int gs = 0;            // this group's tiles (phases of s / sfree / p / pfree)
-    int gd = 0;            // D' sums read by this group
+    int gd = 0;            // D' sums of this group (drained by the two column halves in turn)
     int prev_tok = 0, prev_nvalid = 0;
     bool have_prev = false;
     // add the previous tile's key sums (lane j of this group's D' = key j) to the scores
     auto drain = [&]() -> bool {
       if (!have_prev) return true;
-      const int db = gd & 1;
-      if (!ptx::mbar_wait(&bar_dfull[grp][db], (gd >> 1) & 1, abort, p.status, RC_ETIMEOUT)) return false;
+      have_prev = false;
+      const int db = gd & 1;  // buffer db is drained by column half db
+      const uint32_t phase = (gd >> 1) & 1;
+      ++gd;
+      if (db != ch) return true;
+      if (!ptx::mbar_wait(&bar_dfull[grp][db], phase, abort, p.status, RC_ETIMEOUT)) return false;
       ptx::tc_fence_after();
-      uint32_t r[32];
-      ptx::tmem_ld32(tmem + lane_off + 256 + grp * 32 + db * 16, r);
+      const uint32_t v = ptx::tmem_ld1(tmem + lane_off + 256 + grp * 32 + db * 16);
       ptx::tmem_ld_wait();
-      if (row < prev_nvalid) atomicAdd(p.score_phys + prev_tok + row, __uint_as_float(r[0]));
+      if (row < prev_nvalid) atomicAdd(p.score_phys + prev_tok + row, __uint_as_float(v));
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bar_dfree[grp][db]);
-      ++gd;
-      have_prev = false;
       return true;
     };
     bool ok = true;
@@ -264,37 +295,22 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const __grid_co
           ok = false;
           break;
         }
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t ra[32], rb[32];
-          ptx::tmem_ld32(tS + half * 64, ra);
-          ptx::tmem_ld32(tS + half * 64 + 32, rb);
+        const int lim = t.nvalid - ch * 64;  // valid keys in this half
+        {
+          uint32_t r[32];
+          ptx::tmem_ld32(tS, r);
           ptx::tmem_ld_wait();
-          if (half == 1) {  // S fully read: the MMA may overwrite it
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&bar_sfree[grp]);
-          }
-          uint32_t pk[32];
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const int col = half * 64 + 2 * k;
-            const float a = col < t.nvalid ? ptx::ex2(fmaf(__uint_as_float(ra[2 * k]), c, -lse2)) : 0.f;
-            const float b = col + 1 < t.nvalid ? ptx::ex2(fmaf(__uint_as_float(ra[2 * k + 1]), c, -lse2)) : 0.f;
-            pk[k] = ptx::pack_bf16x2(a, b);
-          }
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const int col = half * 64 + 32 + 2 * k;
-            const float a = col < t.nvalid ? ptx::ex2(fmaf(__uint_as_float(rb[2 * k]), c, -lse2)) : 0.f;
-            const float b = col + 1 < t.nvalid ? ptx::ex2(fmaf(__uint_as_float(rb[2 * k + 1]), c, -lse2)) : 0.f;
-            pk[16 + k] = ptx::pack_bf16x2(a, b);
-          }
-          // P[row][64 half .. 64 half + 63] -> sub-tile `half`, 8 chunks of 16 bytes, swizzled
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-            *reinterpret_cast<uint4*>(sP + half * kSubTileBytes + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
-          }
+          if (lim >= 64) exp_store<false>(r, 0, lim, c, lse2, sProw, row);
+          else exp_store<true>(r, 0, lim, c, lse2, sProw, row);
+        }
+        {
+          uint32_t r[32];
+          ptx::tmem_ld32(tS + 32, r);
+          ptx::tmem_ld_wait();
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(&bar_sfree[grp]);  // S read: the MMA may overwrite it
+          if (lim >= 64) exp_store<false>(r, 32, lim, c, lse2, sProw, row);
+          else exp_store<true>(r, 32, lim, c, lse2, sProw, row);
         }
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(&bar_p[grp]);
