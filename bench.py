@@ -154,9 +154,10 @@ def aggregate_over_ranks(ms: float, work: float, device=None):
     return float(t_max[0]), float(t_sum[0])
 
 
-def make_cfg(w, layers=None):
+def make_cfg(w, layers=None, heads=None):
     from rolling_kv_cache_b200.cache import make_config
-    return make_config(layers=w.layers if layers is None else layers, heads=w.heads,
+    return make_config(layers=w.layers if layers is None else layers,
+                       heads=w.heads if heads is None else heads,
                        head_dim=w.head_dim, grid_h=w.grid_h, grid_w=w.grid_w,
                        sink_frames=w.sink_frames, window_frames=w.window_frames,
                        chunk_frames=w.chunk_frames, policy=w.policy,
@@ -235,6 +236,7 @@ def run_ours(args, w):
     import torch.distributed as dist
     from rolling_kv_cache_b200 import binding as B
     from rolling_kv_cache_b200.cache import RollingKVCache
+    from rolling_kv_cache_b200.shard import head_ranges, sharded_scores_topc
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -245,14 +247,21 @@ def run_ours(args, w):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
 
-    cache = RollingKVCache(make_cfg(w), dev)
+    # --shard heads: this rank owns a head range of one stream (strong scaling);
+    # default: an independent stream per rank (weak scaling)
+    shard = args.shard == "heads"
+    h0, h1 = head_ranges(w.heads, world)[rank] if shard else (0, w.heads)
+    if h1 <= h0:
+        raise SystemExit(f"--shard heads: rank {rank} of {world} would own no head of {w.heads}")
+    cache = RollingKVCache(make_cfg(w, heads=h1 - h0), dev)
     stream = torch.cuda.current_stream(dev)
     # a small pool of distinct seeded inputs, resident in HBM, cycled over
     # (layer, pass, chunk); timing does not depend on the values
     pool = []
     for i in range(6):
-        q, k, v = rc_synth.chunk_qkv(w, i % w.layers, i, i % w.passes, seed=rank)
-        pool.append(tuple(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in (q, k, v)))
+        q, k, v = rc_synth.chunk_qkv(w, i % w.layers, i, i % w.passes, seed=0 if shard else rank)
+        pool.append(tuple(torch.from_numpy(np.ascontiguousarray(x[:, h0:h1]).view(np.int16))
+                          .view(torch.bfloat16).to(dev) for x in (q, k, v)))
     out = torch.empty_like(pool[0][0])
     B_ = w.chunk_frames
     calls_per_step = w.layers * w.passes
@@ -260,14 +269,21 @@ def run_ours(args, w):
     scores = torch.empty(w.footprint_tokens, dtype=torch.float32, device=dev) if w.topc else None
     topc = torch.empty(w.topc, dtype=torch.int32, device=dev) if w.topc else None
 
+    def layer_step(l, q, k, v, frame_start, out_buf):
+        if shard and scores is not None:
+            # this rank's heads only; the score vectors are summed over ranks before top-C
+            cache.step(l, q, k, v, frame_start, out=out_buf, scores=scores)
+            sharded_scores_topc(cache, l, scores, w.topc, topc)
+        else:
+            cache.step(l, q, k, v, frame_start, out=out_buf, scores=scores, topc=topc, C=w.topc)
+
     def run_chunk(c, q_of=None, out_buf=None):
         if c in w.cut_chunks:   # KV flush + RoPE cut before the chunk's first pass
             cache.reindex(w.cut_delta, B.RC_REINDEX_FLUSH | B.RC_REINDEX_CUT)
         for p in range(w.passes):
             for l in range(w.layers):
                 q, k, v = (q_of or pool)[(c * 7 + p * 3 + l) % len(q_of or pool)]
-                cache.step(l, q, k, v, c * B_, out=out if out_buf is None else out_buf,
-                           scores=scores, topc=topc, C=w.topc)
+                layer_step(l, q, k, v, c * B_, out if out_buf is None else out_buf)
 
     chunk = 0
     prefill = (w.footprint_frames + B_ - 1) // B_   # until the window is full
@@ -326,9 +342,14 @@ def run_ours(args, w):
         for p in range(w.passes):
             for l in range(w.layers):
                 q, k, v = host_pool[(p + l) % len(host_pool)]
-                pipe.submit(l, q, k, v, chunk * B_, out_hosts[pipe.i % 2], scores=scores, topc=topc, C=w.topc)
+                if shard and scores is not None:
+                    pipe.submit(l, q, k, v, chunk * B_, out_hosts[pipe.i % 2], scores=scores)
+                    sharded_scores_topc(cache, l, scores, w.topc, topc)
+                else:
+                    pipe.submit(l, q, k, v, chunk * B_, out_hosts[pipe.i % 2], scores=scores, topc=topc,
+                                C=w.topc)
                 st = cache.state(l)
-                e2e_flops += 4.0 * w.head_dim * w.heads * visible_pairs(
+                e2e_flops += 4.0 * w.head_dim * (h1 - h0) * visible_pairs(
                     w, sum(1 for e in st.kept[:st.n_kept] if e.region != 2))
         chunk += 1
     e1 = pipe.record_done()
@@ -358,14 +379,16 @@ def run_ours(args, w):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "strong" if shard else "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
             "config": {"workload": w.name, "layers": w.layers, "heads": w.heads,
                        "head_dim": w.head_dim, "frame_seqlen": w.frame_seqlen,
                        "chunk_frames": B_, "sink_frames": w.sink_frames,
                        "window_frames": w.window_frames, "passes_per_chunk": w.passes,
                        "cached_tokens_per_head": w.footprint_tokens,
                        "step": f"one chunk x {w.layers} layers x {w.passes} passes",
-                       "parallelism": f"independent stream per GPU x{world}",
+                       "parallelism": (f"heads split over {world} GPUs (one stream)" if shard
+                                       else f"independent stream per GPU x{world}"),
                        "l2": "inputs larger than L2 (182 MB K/V ring per layer, 30 layers cycled)"},
             "frames_per_s_per_layer": frames_per_s_per_layer,
             "frames_per_s_model": frames / (ms_max / 1e3),
@@ -422,7 +445,10 @@ def run_hbm(args):
         "inplace": (base.replace(sink_frames=18, window_frames=3), "rerotate", 1),
     }
     res = {}
+    only = [c for c in args.hbm_cases.split(",") if c] if args.hbm_cases else list(cases)
     for name, (w, kind, sink_shift) in cases.items():
+        if name not in only:
+            continue
         cache = RollingKVCache(make_cfg(w, layers=1), dev)
         q, k, v = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
                    for x in rc_synth.chunk_qkv(w, 0, 0, 0))
@@ -466,9 +492,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="wan13b", choices=list(rc_synth.WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--shard", choices=["streams", "heads"], default="streams",
+                    help="streams: an independent stream per rank (weak scaling); heads: each rank "
+                         "owns a head range of one stream, scores summed over ranks before top-C")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (small profiling runs)")
+    ap.add_argument("--hbm-cases", default="",
+                    help="with --hbm: comma list of cases to run (append, rotcopy, inplace; default all)")
     ap.add_argument("--hbm", action="store_true",
                     help="measure the HBM-bound append / re-rotation kernels instead")
     args = ap.parse_args()

@@ -152,6 +152,21 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
                   int frame_start, int n_frames, rc_policy policy, void* out, float* lse,
                   float* scores, int32_t* topc, int C, void* stream);
 
+/* Top-C over a score vector the caller supplies, in the candidate order of
+ * `layer`'s last rc_step. For a stream whose heads are split across GPUs
+ * (each rank's cache holds a head range, and its rc_step scores only those
+ * heads): the ranks sum their score vectors with one all-reduce and select
+ * from the sum. The selection is rc_step's (rCM length-extrapolation guide,
+ * strategy 4, Deep Forcing: keep the candidate tokens with the highest
+ * attention scores): ties to the lower index, output ascending, -1 tail when
+ * there are fewer than C candidates.
+ *   scores: [n_candidates] fp32 device, read only, in rc_step's scores order
+ *     (rc_get_state reports n_candidates).
+ *   topc: [C] int32 device, written: logical indices over the kept list.
+ * Errors: RC_EINVAL (host-only handle, null pointer, C <= 0, bad layer),
+ * RC_ESTATE (no rc_step has run on the layer). Enqueued on `stream`. */
+rc_status rc_select_topc(void* handle, int layer, const float* scores, int C, int32_t* topc, void* stream);
+
 /* rc_step for callers that cannot allocate device memory. The pages have no
  * counterpart; this is a deployment convenience.
  *

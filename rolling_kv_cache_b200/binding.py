@@ -75,7 +75,7 @@ class rc_profile(ctypes.Structure):
 
 
 EXPORTS = ["rc_config_init", "rc_cache_bytes", "rc_cache_create", "rc_step", "rc_step_noalloc",
-           "rc_reindex",
+           "rc_select_topc", "rc_reindex",
            "rc_get_state", "rc_device_status", "rc_rope_table", "rc_cache_layout",
            "rc_watchdog_selftest", "rc_profile_begin", "rc_profile_end", "rc_cache_destroy",
            "rc_last_error"]
@@ -96,6 +96,7 @@ def lib() -> ctypes.CDLL:
         L.rc_cache_create.argtypes = [ctypes.POINTER(rc_config), vp, sz, ctypes.POINTER(vp)]
         L.rc_step.argtypes = [vp, i, vp, vp, vp, i, i, i, vp, vp, vp, vp, i, vp]
         L.rc_step_noalloc.argtypes = L.rc_step.argtypes
+        L.rc_select_topc.argtypes = [vp, i, vp, i, vp, vp]
         L.rc_reindex.argtypes = [vp, i, i, ctypes.c_uint, vp]
         L.rc_get_state.argtypes = [vp, i, ctypes.POINTER(rc_state)]
         L.rc_device_status.argtypes = [vp, vp]
@@ -150,6 +151,11 @@ def rc_step_noalloc(handle, layer, q, k_new, v_new, frame_start, n_frames, polic
     check(lib().rc_step_noalloc(handle, layer, q or None, k_new or None, v_new or None,
                                 frame_start, n_frames, policy, out or None, lse or None,
                                 scores or None, topc or None, C, stream or None))
+
+
+def rc_select_topc(handle, layer, scores, C, topc, stream=0) -> None:
+    """Top-C over a caller-supplied (e.g. rank-summed) score vector in layer's candidate order."""
+    check(lib().rc_select_topc(handle, layer, scores or None, C, topc or None, stream or None))
 
 
 def rc_reindex(handle, policy, t_delta, flags, stream=0) -> None:

@@ -112,6 +112,19 @@ class RollingKVCache:
             return out
         return out_dev
 
+    def select_topc(self, layer: int, scores, C: int, topc=None):
+        """Top-C over ``scores`` ([n_candidates] fp32 on this device, e.g. the
+        sum of the head shards' score vectors) in ``layer``'s candidate order
+        of its last step. Returns ``topc`` ([C] int32)."""
+        if self.device is None:
+            raise ValueError("select_topc needs a device cache")
+        if scores.dtype != torch.float32 or not scores.is_cuda or not scores.is_contiguous():
+            raise ValueError("scores must be a contiguous fp32 device tensor")
+        if topc is None:
+            topc = torch.empty(C, dtype=torch.int32, device=self.device)
+        B.rc_select_topc(self.handle, layer, scores.data_ptr(), C, topc.data_ptr(), self._stream())
+        return topc
+
     def host_pipeline(self, depth: int = 2) -> "HostPipeline":
         """Pipelined stepping from host buffers (see HostPipeline)."""
         return HostPipeline(self, depth)

@@ -191,6 +191,8 @@ struct Cache {
   float* part_o = nullptr;
   float* part_lse = nullptr;
   int sm_count = 148;
+  // candidate frames (slot, logical position) of each layer's last step, for rc_select_topc
+  std::vector<std::vector<std::pair<int, int>>> last_cand;
 };
 
 rc_status check_handle(const void* h) {
@@ -330,6 +332,9 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
   rc::StepPlan plan;
   std::string err;
   if (rc_status st = c->engine->Step(layer, frame_start, n_frames, &plan, &err)) return set_err(st, err);
+  if ((int)c->last_cand.size() < cfg.layers) c->last_cand.resize(cfg.layers);
+  c->last_cand[layer].clear();
+  for (auto& cf : plan.cand) c->last_cand[layer].emplace_back(cf.slot, cf.lpos);
   if (!c->device) return RC_OK;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -518,6 +523,32 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
       if (cudaError_t e = rc::launch_topc(tp, s)) return cuda_err(e, "topc launch");
     }
   }
+  return RC_OK;
+}
+
+rc_status rc_select_topc(void* handle, int layer, const float* scores, int C, int32_t* topc, void* stream) {
+  if (rc_status st = check_handle(handle)) return st;
+  Cache* c = static_cast<Cache*>(handle);
+  if (!c->device) return set_err(RC_EINVAL, "rc_select_topc needs a device handle");
+  if (layer < 0 || layer >= c->cfg.layers) return set_err(RC_EINVAL, "layer out of range");
+  if (!scores || !topc || C <= 0) return set_err(RC_EINVAL, "scores, topc and C > 0 are required");
+  if ((int)c->last_cand.size() <= layer) return set_err(RC_ESTATE, "no step has run on this layer");
+  const auto& cand = c->last_cand[layer];
+  rc::TopCParams tp;
+  std::memset(&tp, 0, sizeof(tp));
+  tp.score_phys = scores;  // already logical: candidate frame i sits at [i F, i F + F)
+  tp.scores_out = c->score_logical;
+  tp.topc = topc;
+  tp.C = C;
+  tp.F = c->cfg.frame_seqlen;
+  tp.n_cand_frames = (int)cand.size();
+  for (size_t i = 0; i < cand.size(); ++i) {
+    tp.cand_slot[i] = (int)i;
+    tp.cand_lpos[i] = cand[i].second;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Timed tm(c->prof, RC_KERNEL_TOPC, s, 0.0, (double)cand.size() * tp.F * 4 * 2);
+  if (cudaError_t e = rc::launch_topc(tp, s)) return cuda_err(e, "topc launch");
   return RC_OK;
 }
 

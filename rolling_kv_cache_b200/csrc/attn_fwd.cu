@@ -7,13 +7,16 @@
 // The mask acts only inside the current chunk (reading M1).
 //
 // One CTA = two 128-query tiles (Q0, Q1) of one head sharing every K/V tile.
-//   warps 0-3   softmax of Q0 (thread = query row = TMEM lane), epilogue
-//   warps 4-7   softmax of Q1, epilogue
-//   warp 8      TMA producer: Q0/Q1 once, K and V into separate 2-stage rings
-//   warp 9      TMEM allocator; one thread issues every tcgen05.mma
+//   warps 0-7   softmax of Q0 and epilogue: 32 query rows (TMEM lanes) x
+//               64 keys per warp, so four softmax warps share each SM
+//               sub-partition's exp2 unit
+//   warps 8-15  softmax of Q1, epilogue
+//   warp 16     TMA producer: Q0/Q1 once, K and V into separate 2-stage rings
+//   warp 17     TMEM allocator; one thread issues every tcgen05.mma
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d), O1 [384,384+d).
-// P_i overwrites the first 64 columns of S_i as packed bf16 and is the A
-// operand of O_i += P_i V.
+// P_i (packed bf16) overwrites columns [0,32) and [64,96) of S_i, each key
+// half in the half of S its softmax warp read, and is the A operand of
+// O_i += P_i V.
 //
 // MMA issue order per KV tile j (FA-style ping-pong):
 //   PV0(j), S0(j+1), PV1(j), S1(j+1)
@@ -38,9 +41,10 @@ namespace rc {
 
 namespace {
 
-constexpr int kFwdThreads = 384;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kSoftmaxWarps = 16;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kFwdThreads = 18 * 32;
 constexpr float kRescaleLog2 = 8.0f;
 
 template <int D>
@@ -148,7 +152,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   using L = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_q, bar_qe, bar_kf[2], bar_vf[2], bar_ke[2], bar_ve[2], bar_s[2], bar_p[2], bar_o[2],
-      bar_fin;
+      bar_fin, bar_pair[8];
+  __shared__ float swap_buf[2][2][2][kTileRows];  // [group][exchange parity][column half][row]
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -165,10 +170,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       ptx::mbar_init(&bar_ke[i], 1);
       ptx::mbar_init(&bar_ve[i], 1);
       ptx::mbar_init(&bar_s[i], 1);
-      ptx::mbar_init(&bar_p[i], 128);
+      ptx::mbar_init(&bar_p[i], 256);
       ptx::mbar_init(&bar_o[i], 1);
     }
     ptx::mbar_init(&bar_fin, 1);
+    for (int i = 0; i < 8; ++i) ptx::mbar_init(&bar_pair[i], 64);
     abort_sh = 0;
     ptx::fence_mbar_init();
   }
@@ -247,9 +253,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     };
     auto issue_pv = [&](int i, int st, bool acc) {
       const uint32_t sV = base_u32 + L::kV + st * L::kTile;
+      // P of keys [16 ks, 16 ks + 16): column (ks / 4) * 64 + (ks % 4) * 8 of S_i
 #pragma unroll
       for (int ks = 0; ks < kTileRows / 16; ++ks)
-        ptx::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + ks * 8,
+        ptx::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + (ks >> 2) * 64 + (ks & 3) * 8,
                     ptx::sdesc_sw128(sV + ks * 2048, kSubTileBytes, 1024), idesc_o, acc || ks > 0);
       ptx::mma_commit(&bar_o[i]);
     };
@@ -300,23 +307,42 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     }
     ptx::mma_commit(&bar_fin);
     ptx::mbar_wait(&bar_fin, 0, noabort, p.status, RC_ETIMEOUT);
-  } else if (warp < 8) {
+  } else if (warp < kSoftmaxWarps) {
     // ---------------------------------------------------------- softmax
-    const int grp = warp >> 2;
+    // group g = warp / 8 owns query tile g. Warp w reads TMEM lane quarter
+    // w % 4 (32 query rows) and column half ch = (w / 4) % 2: keys
+    // [64 ch, 64 ch + 64) of S and output columns [ch D/2, ch D/2 + D/2) of O.
+    // The two warps of a row block (partners) swap their partial row maxima
+    // every tile and their partial row sums once per unit through shared
+    // memory and a 64-thread mbarrier.
+    const int grp = warp >> 3;
+    const int ch = (warp >> 2) & 1;
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + grp * 128;
-    const uint32_t tO = tmem + lane_off + 256 + grp * 128;
+    const uint32_t tS = tmem + lane_off + grp * 128 + ch * 64;
+    const uint32_t tO = tmem + lane_off + 256 + grp * 128 + ch * (D / 2);
+    uint64_t* pbar = &bar_pair[grp * 4 + wq];
     const float c = p.scale_log2;
     const float thresh = kRescaleLog2 / c;
     int gs = 0;  // this group's tiles so far (phase of bar_s / bar_p / bar_o)
+    int nx = 0;  // partner exchanges so far (phase of pbar, slot of swap_buf)
+    // writes v, returns the partner's value (bounded wait)
+    auto swap = [&](float v, float& other) -> bool {
+      float(*buf)[128] = swap_buf[grp][nx & 1];
+      buf[ch][row] = v;
+      ptx::mbar_arrive(pbar);
+      if (!ptx::mbar_wait(pbar, nx & 1, abort, p.status, RC_ETIMEOUT)) return false;
+      ++nx;
+      other = buf[ch ^ 1][row];
+      return true;
+    };
     while (sc.next(jb)) {
       if (*abort) break;
       if (grp == 1 && !jb.has1) continue;
       const int qtok = jb.q0 + grp * kTileRows + row;
       const int my_rank = (min(qtok, p.Nq - 1) / p.F) / p.mask_block;
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
       TileWalker wk{p.seg, p.n_segs, jb.rq_hi};
       wk.seek(jb.kv_lo);
       Tile t;
@@ -325,28 +351,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       for (int j = jb.kv_lo; j < jb.kv_hi && wk.next(t); ++j) {
         if (!ptx::mbar_wait(&bar_s[grp], gs & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
         ptx::tc_fence_after();
-        // columns [0, lim) of this row are visible (the whole row or a ragged tail is masked)
+        // keys [0, lim) of this row are visible (the whole row or a ragged tail is masked);
+        // lim_h of them fall in this warp's half
         const int lim = (t.rank < 0 || t.rank <= my_rank) ? t.nvalid : 0;
-        // pass 1: row maximum of the raw scores (two 32-column loads in flight per wait)
+        const int lim_h = lim - ch * 64;
+        uint32_t ra[32], rb[32];
+        ptx::tmem_ld32(tS, ra);
+        ptx::tmem_ld32(tS + 32, rb);
+        ptx::tmem_ld_wait();
         float mx = -INFINITY;
+        if (lim_h >= 64) {
 #pragma unroll
-        for (int cc = 0; cc < 4; cc += 2) {
-          uint32_t ra[32], rb[32];
-          ptx::tmem_ld32(tS + cc * 32, ra);
-          ptx::tmem_ld32(tS + (cc + 1) * 32, rb);
-          ptx::tmem_ld_wait();
-          if (lim == kTileRows) {
+          for (int k = 0; k < 32; ++k) mx = ptx::fmax3(mx, __uint_as_float(ra[k]), __uint_as_float(rb[k]));
+        } else {
 #pragma unroll
-            for (int k = 0; k < 32; ++k) mx = fmaxf(mx, fmaxf(__uint_as_float(ra[k]), __uint_as_float(rb[k])));
-          } else {
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              mx = fmaxf(mx, cc * 32 + k < lim ? __uint_as_float(ra[k]) : -INFINITY);
-              mx = fmaxf(mx, (cc + 1) * 32 + k < lim ? __uint_as_float(rb[k]) : -INFINITY);
-            }
-          }
+          for (int k = 0; k < 32; ++k)
+            mx = ptx::fmax3(mx, k < lim_h ? __uint_as_float(ra[k]) : -INFINITY,
+                            32 + k < lim_h ? __uint_as_float(rb[k]) : -INFINITY);
         }
-        const float m_new = fmaxf(m, mx);
+        float mo;
+        if (!swap(mx, mo)) { ok = false; break; }
+        const float m_new = ptx::fmax3(m, mx, mo);
         const bool need = m_new > m + thresh;       // also true for the first visible tile
         const bool real = need && m != -INFINITY;   // O already holds weighted values
         if (__any_sync(0xffffffffu, real)) {
@@ -354,7 +379,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           ptx::tc_fence_after();
           const float alpha = real ? ptx::ex2((m - m_new) * c) : 1.f;
 #pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
+          for (int cc = 0; cc < D / 64; ++cc) {
             uint32_t o[32];
             ptx::tmem_ld32(tO + cc * 32, o);
             ptx::tmem_ld_wait();
@@ -367,41 +392,38 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         }
         if (need) m = m_new;
         const float mc = (m == -INFINITY ? 0.f : m) * c;
-        // pass 2: P = 2^(s c - m c), packed bf16 pairs written over S's first
-        // 64 columns; chunk cc's P columns [16cc, 16cc+16) lie in S columns
-        // already read, so the overwrite never races a later read.
+        // P = 2^(s c - m c) as packed bf16 pairs over the first 32 columns of
+        // this half of S (already read): keys 64 ch + 2i, 64 ch + 2i + 1 -> column i
         float sum = 0.f;
-        auto emit = [&](const uint32_t (&r)[32], int cc) {
+        auto emit = [&](const uint32_t (&r)[32], int k0) {
           uint32_t pk[16];
-          if (lim == kTileRows) {
+          if (lim_h >= 64) {
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-              const float a = ptx::ex2(fmaf(__uint_as_float(r[2 * k]), c, -mc));
-              const float b = ptx::ex2(fmaf(__uint_as_float(r[2 * k + 1]), c, -mc));
+              const float a = ptx::ex2_pair(fmaf(__uint_as_float(r[2 * k]), c, -mc), k);
+              const float b = ptx::ex2_pair(fmaf(__uint_as_float(r[2 * k + 1]), c, -mc), k);
               sum += a + b;
               pk[k] = ptx::pack_bf16x2(a, b);
             }
           } else {
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-              const float a = cc * 32 + 2 * k < lim ? ptx::ex2(fmaf(__uint_as_float(r[2 * k]), c, -mc)) : 0.f;
+              const float a = k0 + 2 * k < lim_h ? ptx::ex2_pair(fmaf(__uint_as_float(r[2 * k]), c, -mc), k) : 0.f;
               const float b =
-                  cc * 32 + 2 * k + 1 < lim ? ptx::ex2(fmaf(__uint_as_float(r[2 * k + 1]), c, -mc)) : 0.f;
+                  k0 + 2 * k + 1 < lim_h ? ptx::ex2_pair(fmaf(__uint_as_float(r[2 * k + 1]), c, -mc), k) : 0.f;
               sum += a + b;
               pk[k] = ptx::pack_bf16x2(a, b);
             }
           }
-          ptx::tmem_st16(tS + cc * 16, pk);
+          ptx::tmem_st16(tS + k0 / 2, pk);
         };
-#pragma unroll
-        for (int cc = 0; cc < 4; cc += 2) {
-          uint32_t ra[32], rb[32];
-          ptx::tmem_ld32(tS + cc * 32, ra);
-          ptx::tmem_ld32(tS + (cc + 1) * 32, rb);
-          ptx::tmem_ld_wait();
-          emit(ra, cc);
-          emit(rb, cc + 1);
-        }
+        // S is read again rather than kept in registers across the exchange
+        ptx::tmem_ld32(tS, ra);
+        ptx::tmem_ld_wait();
+        emit(ra, 0);
+        ptx::tmem_ld32(tS + 32, rb);
+        ptx::tmem_ld_wait();
+        emit(rb, 32);
         ptx::tmem_st_wait();
         l += sum;
         ptx::tc_fence_before();
@@ -410,15 +432,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         ++done;
       }
       // epilogue: O / l, to the output (bf16 [Nq][H][D], lse in natural log)
-      // or to this CTA's partial slot (fp32, log2-sum-exp)
+      // or to this CTA's partial slot (fp32, log2-sum-exp); each warp writes
+      // its D/2 columns
+      float l_other = 0.f;
+      if (ok && !swap(l, l_other)) ok = false;
+      const float lt = l + l_other;
       const bool have_o =
           ok && done > 0 && ptx::mbar_wait(&bar_o[grp], (gs - 1) & 1, abort, p.status, RC_ETIMEOUT);
       ptx::tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      const float lse2 = l > 0.f ? m * c + __log2f(l) : -INFINITY;
+      const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
+      const float lse2 = lt > 0.f ? m * c + __log2f(lt) : -INFINITY;
       const int prow = grp * kTileRows + row;
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int cc = 0; cc < D / 64; ++cc) {
         uint32_t o[32];
         if (have_o) {
           ptx::tmem_ld32(tO + cc * 32, o);
@@ -428,8 +454,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           for (int k = 0; k < 32; ++k) o[k] = 0u;
         }
         if (qtok >= p.Nq) continue;
+        const int col = ch * (D / 2) + cc * 32;
         if (jb.slot < 0) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)qtok * p.H + jb.h) * D + cc * 32);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)qtok * p.H + jb.h) * D + col);
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 u;
@@ -440,14 +467,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
             dst[v] = u;
           }
         } else {
-          float4* dst = reinterpret_cast<float4*>(p.part_o + ((size_t)jb.slot * 2 * kTileRows + prow) * D + cc * 32);
+          float4* dst = reinterpret_cast<float4*>(p.part_o + ((size_t)jb.slot * 2 * kTileRows + prow) * D + col);
 #pragma unroll
           for (int v = 0; v < 8; ++v)
             dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
                                  __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
         }
       }
-      if (qtok < p.Nq) {
+      if (qtok < p.Nq && ch == 0) {
         if (jb.slot < 0) {
           if (p.lse) p.lse[(size_t)jb.h * p.Nq + qtok] = lse2 * 0.69314718055994531f;
         } else {
