@@ -400,17 +400,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           if (lim_h >= 64) {
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-              const float a = ptx::ex2_pair(fmaf(__uint_as_float(r[2 * k]), c, -mc), k);
-              const float b = ptx::ex2_pair(fmaf(__uint_as_float(r[2 * k + 1]), c, -mc), k);
+              const float a = ptx::ex2(fmaf(__uint_as_float(r[2 * k]), c, -mc));
+              const float b = ptx::ex2(fmaf(__uint_as_float(r[2 * k + 1]), c, -mc));
               sum += a + b;
               pk[k] = ptx::pack_bf16x2(a, b);
             }
           } else {
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-              const float a = k0 + 2 * k < lim_h ? ptx::ex2_pair(fmaf(__uint_as_float(r[2 * k]), c, -mc), k) : 0.f;
+              const float a = k0 + 2 * k < lim_h ? ptx::ex2(fmaf(__uint_as_float(r[2 * k]), c, -mc)) : 0.f;
               const float b =
-                  k0 + 2 * k + 1 < lim_h ? ptx::ex2_pair(fmaf(__uint_as_float(r[2 * k + 1]), c, -mc), k) : 0.f;
+                  k0 + 2 * k + 1 < lim_h ? ptx::ex2(fmaf(__uint_as_float(r[2 * k + 1]), c, -mc)) : 0.f;
               sum += a + b;
               pk[k] = ptx::pack_bf16x2(a, b);
             }

@@ -206,39 +206,12 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// 2^x on the FMA pipe, to take part of the exponentials off the SFU: x =
-// n + f with n = rint(x) (adding 1.5 * 2^23 rounds to an integer held in the
-// low mantissa bits), f in [-0.5, 0.5]; 2^f by a cubic fitted for minimax
-// relative error on that interval by Lawson's iteration (max relative error
-// 7.5e-5, far below a bf16 half-ulp); n is added to the exponent field.
-// x >= -126 after the clamp, so the exponent field stays >= 0.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = __fadd_rn(x, 12582912.f);
-  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
-  float p = fmaf(0.05517132f, f, 0.24261054f);
-  p = fmaf(p, f, 0.69326097f);
-  p = fmaf(p, f, 0.99992812f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-// The softmax loops run every kExp2FmaEvery-th pair of exponentials on the
-// FMA pipe and the rest on the SFU (0 = all on the SFU); k is the pair index
-// of an unrolled loop, so the choice is made at compile time.
-#ifndef RC_EXP2_FMA_EVERY
-#define RC_EXP2_FMA_EVERY 0
-#endif
-constexpr int kExp2FmaEvery = RC_EXP2_FMA_EVERY;
-__device__ __forceinline__ float ex2_pair(float x, int k) {
-  if (kExp2FmaEvery > 0 && k % (kExp2FmaEvery > 0 ? kExp2FmaEvery : 1) == kExp2FmaEvery - 1) return exp2_fma(x);
-  return ex2(x);
-}
 
 }  // namespace ptx
 }  // namespace rc

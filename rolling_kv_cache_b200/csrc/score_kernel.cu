@@ -91,8 +91,8 @@ __device__ __forceinline__ void exp_store(const uint32_t (&r)[32], int c0, int l
   uint32_t pk[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
-    float a = ptx::ex2_pair(fmaf(__uint_as_float(r[2 * k]), c, -lse2), k);
-    float b = ptx::ex2_pair(fmaf(__uint_as_float(r[2 * k + 1]), c, -lse2), k);
+    float a = ptx::ex2(fmaf(__uint_as_float(r[2 * k]), c, -lse2));
+    float b = ptx::ex2(fmaf(__uint_as_float(r[2 * k + 1]), c, -lse2));
     if (kCheck) {
       if (c0 + 2 * k >= lim) a = 0.f;
       if (c0 + 2 * k + 1 >= lim) b = 0.f;
