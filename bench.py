@@ -57,7 +57,9 @@ def attention_flops(w, n_hist_frames: int, heads=None) -> float:
 
 
 def steady_hist_frames(w) -> int:
-    return w.footprint_frames - w.chunk_frames
+    """Frames' worth of cached keys besides the chunk at steady state (the
+    Deep Forcing region counts as budget / F frames)."""
+    return w.footprint_tokens // w.frame_seqlen - w.chunk_frames
 
 
 def load_peaks():
@@ -164,7 +166,9 @@ def make_cfg(w, layers=None, heads=None):
                        mask_block_frames=w.mask_block_frames, theta=w.theta, t_max=w.t_max,
                        rs_bank_blocks=w.rs_bank_blocks, rs_sink_blocks=w.rs_sink_blocks,
                        rs_static_semantics=w.rs_static_semantics, ir_f_limit=w.ir_f_limit,
-                       ir_sink_blocks=w.ir_sink_blocks, ir_cache_blocks=w.ir_cache_blocks)
+                       ir_sink_blocks=w.ir_sink_blocks, ir_cache_blocks=w.ir_cache_blocks,
+                       df_budget_tokens=w.df_budget_tokens, rf_history_frames=w.rf_history_frames,
+                       rf_weight=w.rf_weight)
 
 
 # ------------------------------------------------------------ CPU oracle
@@ -173,13 +177,15 @@ def oracle_sample_seconds(w, heads: int, chunk: int = 7):
     restricted to ``heads`` heads. Returns (seconds, flops, threads)."""
     from oracle import OracleStream
     st = OracleStream(w, layer=0, seed=0)
+    rng = np.random.default_rng(0)   # Deep Forcing: the oracle's region follows given scores
     for c in range(chunk + 1):
-        st.step(c, w.passes - 1 if c < chunk else 0)
+        pool = rng.random(st.df.next_pool_size(w.chunk_frames)) if st.df is not None else None
+        st.step(c, w.passes - 1 if c < chunk else 0, **({"pool_scores": pool} if st.df is not None else {}))
     st.outputs(heads=[0], rows=np.arange(1))       # warm the regenerated inputs
     t0 = time.perf_counter()
     st.outputs(heads=list(range(heads)))
     dt = time.perf_counter() - t0
-    n_hist = sum(1 for k in st.kept if k.region != "cur")
+    n_hist = sum(1 for k in st.kept_tokens if k.region != "cur") // w.frame_seqlen
     try:
         from threadpoolctl import threadpool_info
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
@@ -318,6 +324,8 @@ def run_ours(args, w):
     prof = B.rc_profile_end(cache.handle)
     cache.device_status()
 
+    # bytes of one layer's K and V buffers (ring, plus the Deep Forcing region)
+    kv_ring_mb = 2 * (h1 - h0) * w.footprint_tokens * w.head_dim * 2 / 1e6
     att = prof["attention"]
     ms_max, flops_total = aggregate_over_ranks(ms, att["flops"], dev)
     value = flops_total / (ms_max / 1e3) / 1e12
@@ -350,7 +358,7 @@ def run_ours(args, w):
                                 C=w.topc)
                 st = cache.state(l)
                 e2e_flops += 4.0 * w.head_dim * (h1 - h0) * visible_pairs(
-                    w, sum(1 for e in st.kept[:st.n_kept] if e.region != 2))
+                    w, sum(1 for e in st.kept[:st.n_kept] if e.region != 2) + st.comp_tokens // w.frame_seqlen)
         chunk += 1
     e1 = pipe.record_done()
     torch.cuda.synchronize()
@@ -389,7 +397,8 @@ def run_ours(args, w):
                        "step": f"one chunk x {w.layers} layers x {w.passes} passes",
                        "parallelism": (f"heads split over {world} GPUs (one stream)" if shard
                                        else f"independent stream per GPU x{world}"),
-                       "l2": "inputs larger than L2 (182 MB K/V ring per layer, 30 layers cycled)"},
+                       "l2": (f"inputs larger than L2 ({kv_ring_mb:.0f} MB K/V ring per layer"
+                              f"{', %d layers cycled' % w.layers if w.layers > 1 else ''})")},
             "frames_per_s_per_layer": frames_per_s_per_layer,
             "frames_per_s_model": frames / (ms_max / 1e3),
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,

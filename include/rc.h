@@ -23,7 +23,10 @@
  *   - rCM length-extrapolation guide (dpshk.com), strategies 1-3: sliding
  *     window with sink blocks, Rolling Sink, Infinity-RoPE (block-relative
  *     time, clamp at 0, KV flush, RoPE cut); the cache bound is computed up
- *     front and preallocated.
+ *     front and preallocated. Strategy 4, Deep Forcing (deep sink + top-C
+ *     tokens by attention score + recent tail, time encodings rewritten so no
+ *     holes remain) and strategy 5, Relax Forcing (sink + history frames
+ *     chosen by w * alignment + (1 - w) * complementarity + tail).
  *   - Rolling Sink digest (paper.rainbus.top/paper/2602.07775), method-step
  *     details: sink time indices slide to [i-K, i-(K-S)); sink content is a
  *     length-S segment of Roll(x_[0,K)), forward on even cycles, reversed on
@@ -70,7 +73,11 @@ typedef enum rc_policy {
   RC_NONE = 0,           /* unbounded baseline: keep every frame (capacity must cover the video) */
   RC_SLIDING = 1,        /* sliding window + attention sink (rCM strategy 1, LingBot) */
   RC_ROLLING_SINK = 2,   /* Rolling Sink: bank roll + sliding sink time indices */
-  RC_INFINITY_ROPE = 3   /* Infinity-RoPE: block-relative time, clamp at 0, flush + cut */
+  RC_INFINITY_ROPE = 3,  /* Infinity-RoPE: block-relative time, clamp at 0, flush + cut */
+  RC_DEEP_FORCING = 4,   /* Deep Forcing: deep sink + top-C scored tokens + recent tail
+                            (rCM length-extrapolation guide, strategy 4); see below */
+  RC_RELAX_FORCING = 5   /* Relax Forcing: sink + K history frames chosen by cosine
+                            similarity + recent tail (strategy 5); see below */
 } rc_policy;
 
 /* rc_reindex flags */
@@ -105,7 +112,41 @@ typedef struct rc_config {
   int ir_sink_blocks;     /* Infinity-RoPE: global sink blocks (sink_frames = this * chunk_frames) */
   int ir_cache_blocks;    /* Infinity-RoPE: blocks kept before the current one, sink included
                              (window_frames = (cache - sink + 1) * chunk_frames) */
+  int df_budget_tokens;   /* Deep Forcing: tokens of the compressed region (a multiple of
+                             frame_seqlen); sink_frames = deep sink, window_frames = recent
+                             tail including the current chunk (>= 2 chunks) */
+  int rf_history_frames;  /* Relax Forcing: K, history frames kept between sink and tail */
+  double rf_weight;       /* Relax Forcing: w in score = w * alignment + (1 - w) * complement */
 } rc_config;
+
+/* Relax Forcing (rCM length-extrapolation guide, strategy 5): the cache keeps
+ * the sink (the first sink_frames frames), at most rf_history_frames history
+ * frames and the recent tail (the newest window_frames frames up to the
+ * current chunk's end). When a new chunk pushes the tail's oldest frames out
+ * they join the history frames in a pool; if the pool holds more than K frames
+ * the K with the highest score = w * alignment + (1 - w) * complement stay
+ * (ties to the older frame), in time order. A frame's descriptor is the mean
+ * over its tokens of its raw key, heads concatenated; alignment = cosine with
+ * the mean descriptor of the tail (the new chunk included); complement = 1 -
+ * the mean cosine with the other pool frames. Every frame keeps its own
+ * absolute time index (nothing is re-rotated). Chunks are whole blocks. */
+
+/* Deep Forcing (rCM length-extrapolation guide, strategy 4): the cache keeps
+ * the deep sink (the first sink_frames frames), a compressed region of at most
+ * df_budget_tokens tokens chosen by attention score, and the recent tail (the
+ * newest window_frames frames up to the current chunk's end). Every rc_step
+ * scores the cached tokens (the softmax mass each key receives, summed over
+ * heads and queries, as rc_step's scores output). When a new chunk pushes the
+ * tail's oldest frames out, they join the compressed region's tokens in a pool
+ * and the df_budget_tokens highest-scoring pool tokens (scores of the last
+ * step before the chunk, ties to the lower index) form the new region, in
+ * time order. Time indices leave no holes: tail and chunk frames keep tau = g;
+ * with g_t the first tail frame and V = region tokens / frame_seqlen, region
+ * token i has tau = g_t - V + i / frame_seqlen and sink frame j has
+ * tau = g_t - V - sink_frames + j, so sink, region and tail sit on
+ * consecutive time positions; the region's and the sink's keys are rotated to
+ * their new times on the device (the page's in-place rope_time_delta_).
+ * Chunks are whole blocks of chunk_frames frames. */
 
 /* Fill *cfg with defaults for the pages' short signature
  * (layers, heads, head_dim, frame_seqlen, sink_frames, window_frames):
@@ -229,10 +270,30 @@ typedef struct rc_state {
   int32_t evicted[RC_MAX_SLOTS];  /* contents that left the cache at the last new chunk */
   int32_t n_evicted;
   rc_frame_state kept[RC_MAX_SLOTS];
+  int32_t comp_tokens;       /* Deep / Relax Forcing: tokens in the selected region (logically
+                                between the sink and the tail frames; 0 for other policies) */
+  int32_t comp_tau0;         /* Deep Forcing: region token i has tau = comp_tau0 + i / frame_seqlen;
+                                Relax Forcing: -1 (each region frame keeps its own index) */
+  int32_t comp_row0;         /* Deep / Relax Forcing: physical row (per head) of region token 0 in the K/V
+                                buffers (rows past the ring: (sink + window) * F + b * budget) */
 } rc_state;
 
 /* Copy a layer's cache state (after its last rc_step) to host memory. */
 rc_status rc_get_state(const void* handle, int layer, rc_state* out);
+
+/* Deep Forcing / Relax Forcing: the source of each token of a layer's
+ * selected region (Deep Forcing's compressed tokens, Relax Forcing's history
+ * frames), in region order: frame[i] = stream frame, tok[i] = token index in
+ * that frame (row-major h, w). frame and tok are host arrays of at least
+ * rc_state.comp_tokens entries. Synchronizes `stream` (the selection lives on
+ * the device). RC_EINVAL for other policies or a host-only handle. */
+rc_status rc_comp_tokens(void* handle, int layer, int32_t* frame, int32_t* tok, void* stream);
+
+/* Relax Forcing: the pool scores of a layer's last selection (pool order:
+ * history frames, then the frames that left the tail), to host memory.
+ * *n receives the pool size (0 if the last new chunk needed no selection);
+ * scores must hold RC_MAX_SLOTS floats. Synchronizes `stream`. */
+rc_status rc_pool_scores(void* handle, int layer, float* scores, int32_t* n, void* stream);
 
 /* Synchronize `stream` and report the device-side status word: RC_OK, or
  * RC_ETIMEOUT if a kernel's bounded wait gave up since the last check
@@ -247,8 +308,10 @@ rc_status rc_rope_table(const void* handle, int axis, float* dst, size_t* count)
 
 typedef struct rc_layout {
   size_t kv_layer_stride;  /* bytes between one layer's K and the next layer's K */
-  size_t k_offset;         /* layer 0's K ring buffer [heads][capacity][head_dim] bf16 */
-  size_t v_offset;         /* layer 0's V ring buffer, same shape */
+  size_t k_offset;         /* layer 0's K ring buffer [heads][head_dim/64][capacity][64] bf16:
+                              each head in 64-dim planes (dims 64p .. 64p+63 of token t at
+                              plane p, row t) */
+  size_t v_offset;         /* layer 0's V ring buffer, same layout */
   size_t raw_layer_stride; /* bytes between layers of the pristine source */
   size_t raw_k_offset;     /* pristine raw K [heads][raw_frames*F][head_dim] (0 if none) */
   size_t raw_v_offset;     /* pristine raw V (Rolling Sink bank, 0 if none) */
@@ -277,7 +340,8 @@ rc_status rc_watchdog_selftest(void* handle, unsigned limit_us, void* stream);
  * the summed device milliseconds, then disarms. Launches beyond the limit
  * are counted but not timed. */
 enum { RC_KERNEL_REROTATE = 0, RC_KERNEL_APPEND = 1, RC_KERNEL_ATTENTION = 2,
-       RC_KERNEL_SCORES = 3, RC_KERNEL_TOPC = 4, RC_KERNEL_COMBINE = 5, RC_KERNEL_KINDS = 6 };
+       RC_KERNEL_SCORES = 3, RC_KERNEL_TOPC = 4, RC_KERNEL_COMBINE = 5, RC_KERNEL_COMPACT = 6,
+       RC_KERNEL_KINDS = 7 };
 typedef struct rc_profile {
   int64_t launches[RC_KERNEL_KINDS];
   int64_t timed[RC_KERNEL_KINDS];

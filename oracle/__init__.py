@@ -32,10 +32,11 @@ invariants, torch's SDPA, brute force). See tests/test_oracle_*.py.
 from .policy import PolicyOracle, KeptFrame, roll_index
 from .rope import rope_pair_split, rope_angles, rope_apply, token_grid_positions
 from .attention import masked_sdpa, visibility, column_scores, top_c
+from .deep_forcing import DeepForcingOracle, KeptToken
 from .stream import OracleStream
 
 __all__ = [
     "PolicyOracle", "KeptFrame", "roll_index", "rope_pair_split", "rope_angles",
     "rope_apply", "token_grid_positions", "masked_sdpa", "visibility",
-    "column_scores", "top_c", "OracleStream",
+    "column_scores", "top_c", "OracleStream", "DeepForcingOracle", "KeptToken",
 ]

@@ -15,7 +15,9 @@ from typing import Dict, List, Optional, Sequence
 import numpy as np
 
 import rc_synth
-from .policy import KeptFrame, PolicyOracle
+from .policy import POLICY_DEEP_FORCING, POLICY_RELAX_FORCING, KeptFrame, PolicyOracle
+from .deep_forcing import DeepForcingOracle, KeptToken
+from .relax_forcing import RelaxForcingOracle, frame_descriptor
 from .rope import rope_angles, rope_apply, token_grid_positions
 from .attention import column_scores, masked_sdpa, top_c, visibility
 
@@ -28,23 +30,53 @@ class OracleStream:
         self.w = w
         self.layer = layer
         self.seed = seed
-        self.policy = PolicyOracle.from_workload(w)
+        self.df = self.rf = None
+        if w.policy == POLICY_DEEP_FORCING:
+            self.policy = None
+            self.df = DeepForcingOracle(w.chunk_frames, w.sink_frames, w.window_frames,
+                                        w.df_budget_tokens, w.frame_seqlen)
+        elif w.policy == POLICY_RELAX_FORCING:
+            self.policy = self.rf = RelaxForcingOracle(
+                w.chunk_frames, w.sink_frames, w.window_frames, w.rf_history_frames, w.rf_weight,
+                lambda g: frame_descriptor(self.frame_raw(g, rc_synth.TENSOR_K)))
+        else:
+            self.policy = PolicyOracle.from_workload(w)
         self.last_pass: Dict[int, int] = {}
         self.cur = None
         self.kept: List[KeptFrame] = []
+        self.kept_tokens: List[KeptToken] = []
         self._lru: "OrderedDict[tuple, np.ndarray]" = OrderedDict()
         self._lru_cap = 3 * cache_chunks
 
     # ------------------------------------------------------------ stream
     def reindex(self, flags: int, t_delta: int) -> None:
+        if self.df is not None:
+            raise ValueError("Deep Forcing has no reindex operation")
         self.policy.reindex(flags, t_delta)
 
-    def step(self, chunk: int, pass_: int) -> List[KeptFrame]:
+    def step(self, chunk: int, pass_: int, pool_scores=None, selection=None):
+        """Advance the policy; returns the kept frames (the kept key tokens
+        under Deep Forcing, which takes the pool's scores or selection at a
+        compaction: see DeepForcingOracle.step; Relax Forcing takes an
+        optional selection, see RelaxForcingOracle.step)."""
         B = self.w.chunk_frames
-        self.kept = self.policy.step(chunk * B, B)
+        # this pass's raw values are what the cache holds from now on (D1)
         self.last_pass[chunk] = pass_
+        if self.df is not None:
+            self.kept_tokens = self.df.step(chunk * B, B, pool_scores, selection)
+            self.kept = []
+        elif self.rf is not None:
+            self.kept = self.rf.step(chunk * B, B, selection)
+            F = self.w.frame_seqlen
+            self.kept_tokens = [KeptToken(k.content, t, k.tau, k.region, k.rank)
+                                for k in self.kept for t in range(F)]
+        else:
+            self.kept = self.policy.step(chunk * B, B)
+            F = self.w.frame_seqlen
+            self.kept_tokens = [KeptToken(k.content, t, k.tau, k.region, k.rank)
+                                for k in self.kept for t in range(F)]
         self.cur = (chunk, pass_)
-        return self.kept
+        return self.kept_tokens if self.df is not None else self.kept
 
     # ------------------------------------------------------------ inputs
     def tensor(self, chunk: int, pass_: int, tid: int) -> np.ndarray:
@@ -67,15 +99,28 @@ class OracleStream:
         return t[o * F:(o + 1) * F]
 
     # ----------------------------------------------------------- outputs
-    def key_layout(self, kept: Optional[Sequence[KeptFrame]] = None):
-        """Per logical key token: tau, mask rank, region code (0 sink, 1 hist, 2 cur)."""
-        kept = self.kept if kept is None else kept
-        F = self.w.frame_seqlen
-        tau = np.repeat([k.tau for k in kept], F)
-        rank = np.repeat([k.rank for k in kept], F)
-        code = {"sink": 0, "hist": 1, "cur": 2}
-        region = np.repeat([code[k.region] for k in kept], F)
+    def key_layout(self):
+        """Per logical key token: tau, mask rank, region code (0 sink, 1
+        history: compressed region and tail before the chunk, 2 current)."""
+        kt = self.kept_tokens
+        code = {"sink": 0, "comp": 1, "hist": 1, "cur": 2}
+        tau = np.array([k.tau for k in kt], dtype=np.int64)
+        rank = np.array([k.rank for k in kt], dtype=np.int64)
+        region = np.array([code[k.region] for k in kt], dtype=np.int64)
         return tau, rank, region
+
+    def _key_raw(self, tid: int) -> np.ndarray:
+        """Raw k or v of every kept key token, in logical order."""
+        kt = self.kept_tokens
+        out, i = [], 0
+        while i < len(kt):   # runs of tokens of one frame, gathered at once
+            j = i
+            while j + 1 < len(kt) and kt[j + 1].content == kt[i].content and kt[j + 1].region == kt[i].region:
+                j += 1
+            toks = np.array([k.tok for k in kt[i:j + 1]])
+            out.append(self.frame_raw(kt[i].content, tid)[toks])
+            i = j + 1
+        return np.concatenate(out)
 
     def outputs(self, heads: Optional[Sequence[int]] = None,
                 rows: Optional[np.ndarray] = None, want_scores: bool = False):
@@ -94,16 +139,15 @@ class OracleStream:
         if want_scores and len(rows) != nq:
             raise ValueError("scores need every query row")
         hh, ww = token_grid_positions(F, w.grid_w)
-        cur_tau = {k.rank: k.tau for k in self.kept if k.region == "cur"}
+        cur_tau = {k.rank: k.tau for k in self.kept_tokens if k.region == "cur"}
         q_raw = self.tensor(chunk, pass_, rc_synth.TENSOR_Q)[rows]
         q_tau = np.array([cur_tau[r // F] for r in rows])
         q_rot = rope_apply(q_raw, rope_angles(q_tau, hh[rows % F], ww[rows % F], d, w.theta))
 
         k_tau, k_rank, region = self.key_layout()
-        k_raw = np.concatenate([self.frame_raw(k.content, rc_synth.TENSOR_K) for k in self.kept])
-        v_raw = np.concatenate([self.frame_raw(k.content, rc_synth.TENSOR_V) for k in self.kept])
-        nk = k_raw.shape[0]
-        tok = np.arange(nk) % F
+        k_raw = self._key_raw(rc_synth.TENSOR_K)
+        v_raw = self._key_raw(rc_synth.TENSOR_V)
+        tok = np.array([k.tok for k in self.kept_tokens])
         k_rot = rope_apply(k_raw, rope_angles(k_tau, hh[tok], ww[tok], d, w.theta))
         vis = visibility(rows // F, k_rank, w.mask_block_frames)
 

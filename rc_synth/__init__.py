@@ -24,6 +24,8 @@ import numpy as np
 TENSOR_Q, TENSOR_K, TENSOR_V = 0, 1, 2
 
 POLICY_NONE, POLICY_SLIDING, POLICY_ROLLING_SINK, POLICY_INFINITY_ROPE = 0, 1, 2, 3
+POLICY_DEEP_FORCING = 4
+POLICY_RELAX_FORCING = 5
 
 
 @dataclasses.dataclass(frozen=True)
@@ -56,6 +58,11 @@ class Workload:
     cut_delta: int = 0
     # per-token scores + top-C on every step (0 = off)
     topc: int = 0
+    # Deep Forcing: compressed-region budget in tokens (a multiple of the frame size)
+    df_budget_tokens: int = 0
+    # Relax Forcing: history frames kept between sink and tail, alignment weight
+    rf_history_frames: int = 0
+    rf_weight: float = 0.5
     mask_block_frames: int = 1
     theta: float = 10000.0
     t_max: int = 4096
@@ -74,7 +81,7 @@ class Workload:
 
     @property
     def footprint_tokens(self) -> int:
-        return self.footprint_frames * self.frame_seqlen
+        return (self.footprint_frames + self.rf_history_frames) * self.frame_seqlen + self.df_budget_tokens
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -106,6 +113,21 @@ WORKLOADS = {
         policy=POLICY_INFINITY_ROPE, chunks=100, passes=1, dist="normal",
         ir_f_limit=21, ir_sink_blocks=1, ir_cache_blocks=6,
         cut_chunks=(27, 60), cut_delta=21, topc=4680),
+    # Deep Forcing (rCM page, strategy 4): deep sink 3 frames + a compressed
+    # region of 12 frames' worth of tokens + recent tail of 6 frames (current
+    # chunk included); same 32760-token footprint as the two block policies.
+    "deep_forcing": Workload(
+        name="deep_forcing", workload_id=6, layers=1, heads=12, head_dim=128,
+        grid_h=30, grid_w=52, chunk_frames=3, sink_frames=3, window_frames=6,
+        policy=POLICY_DEEP_FORCING, chunks=60, passes=1, dist="normal",
+        df_budget_tokens=12 * 1560),
+    # Relax Forcing (rCM page, strategy 5): sink 3 frames + 12 history frames
+    # chosen by cosine similarity + tail of 6 frames; same 32760-token footprint.
+    "relax_forcing": Workload(
+        name="relax_forcing", workload_id=7, layers=1, heads=12, head_dim=128,
+        grid_h=30, grid_w=52, chunk_frames=3, sink_frames=3, window_frames=6,
+        policy=POLICY_RELAX_FORCING, chunks=60, passes=1, dist="normal_frame_mean",
+        rf_history_frames=12, rf_weight=0.5),
 }
 
 

@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "librc.so")
 
 RC_OK, RC_EINVAL, RC_ESTATE, RC_ECUDA, RC_ERANGE, RC_ETIMEOUT, RC_ENOMEM = range(7)
-RC_NONE, RC_SLIDING, RC_ROLLING_SINK, RC_INFINITY_ROPE = range(4)
+RC_NONE, RC_SLIDING, RC_ROLLING_SINK, RC_INFINITY_ROPE, RC_DEEP_FORCING, RC_RELAX_FORCING = range(6)
 RC_REINDEX_FLUSH, RC_REINDEX_CUT, RC_REINDEX_SINK = 1, 2, 4
 RC_MAX_SLOTS = 256
 RC_MAX_CHUNK_FRAMES = 16
@@ -38,6 +38,8 @@ class rc_config(ctypes.Structure):
         ("rs_bank_blocks", ctypes.c_int), ("rs_sink_blocks", ctypes.c_int),
         ("rs_static_semantics", ctypes.c_int), ("ir_f_limit", ctypes.c_int),
         ("ir_sink_blocks", ctypes.c_int), ("ir_cache_blocks", ctypes.c_int),
+        ("df_budget_tokens", ctypes.c_int), ("rf_history_frames", ctypes.c_int),
+        ("rf_weight", ctypes.c_double),
     ]
 
 
@@ -54,6 +56,7 @@ class rc_state(ctypes.Structure):
         ("n_candidates", ctypes.c_int32), ("n_jobs", ctypes.c_int32),
         ("evicted", ctypes.c_int32 * RC_MAX_SLOTS), ("n_evicted", ctypes.c_int32),
         ("kept", rc_frame_state * RC_MAX_SLOTS),
+        ("comp_tokens", ctypes.c_int32), ("comp_tau0", ctypes.c_int32), ("comp_row0", ctypes.c_int32),
     ]
 
 
@@ -65,17 +68,18 @@ class rc_layout(ctypes.Structure):
                 ("raw_frames", ctypes.c_int32), ("total", ctypes.c_size_t)]
 
 
-RC_KERNEL_NAMES = ["rerotate", "append", "attention", "scores", "topc", "combine"]
+RC_KERNEL_NAMES = ["rerotate", "append", "attention", "scores", "topc", "combine", "compact"]
+_NK = len(RC_KERNEL_NAMES)
 
 
 class rc_profile(ctypes.Structure):
-    _fields_ = [("launches", ctypes.c_int64 * 6), ("timed", ctypes.c_int64 * 6),
-                ("ms", ctypes.c_double * 6), ("flops", ctypes.c_double * 6),
-                ("bytes", ctypes.c_double * 6)]
+    _fields_ = [("launches", ctypes.c_int64 * _NK), ("timed", ctypes.c_int64 * _NK),
+                ("ms", ctypes.c_double * _NK), ("flops", ctypes.c_double * _NK),
+                ("bytes", ctypes.c_double * _NK)]
 
 
 EXPORTS = ["rc_config_init", "rc_cache_bytes", "rc_cache_create", "rc_step", "rc_step_noalloc",
-           "rc_select_topc", "rc_reindex",
+           "rc_select_topc", "rc_reindex", "rc_comp_tokens", "rc_pool_scores",
            "rc_get_state", "rc_device_status", "rc_rope_table", "rc_cache_layout",
            "rc_watchdog_selftest", "rc_profile_begin", "rc_profile_end", "rc_cache_destroy",
            "rc_last_error"]
@@ -97,6 +101,8 @@ def lib() -> ctypes.CDLL:
         L.rc_step.argtypes = [vp, i, vp, vp, vp, i, i, i, vp, vp, vp, vp, i, vp]
         L.rc_step_noalloc.argtypes = L.rc_step.argtypes
         L.rc_select_topc.argtypes = [vp, i, vp, i, vp, vp]
+        L.rc_comp_tokens.argtypes = [vp, i, vp, vp, vp]
+        L.rc_pool_scores.argtypes = [vp, i, vp, vp, vp]
         L.rc_reindex.argtypes = [vp, i, i, ctypes.c_uint, vp]
         L.rc_get_state.argtypes = [vp, i, ctypes.POINTER(rc_state)]
         L.rc_device_status.argtypes = [vp, vp]
@@ -156,6 +162,22 @@ def rc_step_noalloc(handle, layer, q, k_new, v_new, frame_start, n_frames, polic
 def rc_select_topc(handle, layer, scores, C, topc, stream=0) -> None:
     """Top-C over a caller-supplied (e.g. rank-summed) score vector in layer's candidate order."""
     check(lib().rc_select_topc(handle, layer, scores or None, C, topc or None, stream or None))
+
+
+def rc_comp_tokens(handle, layer, n, stream=0):
+    """Deep Forcing: (frames, tokens) int32 arrays of the layer's compressed region."""
+    frame = (ctypes.c_int32 * max(1, n))()
+    tok = (ctypes.c_int32 * max(1, n))()
+    check(lib().rc_comp_tokens(handle, layer, frame, tok, stream or None))
+    return list(frame)[:n], list(tok)[:n]
+
+
+def rc_pool_scores(handle, layer, stream=0):
+    """Relax Forcing: the pool scores of the layer's last frame selection."""
+    buf = (ctypes.c_float * RC_MAX_SLOTS)()
+    n = ctypes.c_int32()
+    check(lib().rc_pool_scores(handle, layer, buf, ctypes.byref(n), stream or None))
+    return list(buf)[:n.value]
 
 
 def rc_reindex(handle, policy, t_delta, flags, stream=0) -> None:

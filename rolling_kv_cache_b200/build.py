@@ -13,6 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "librc.so")
 SOURCES = ["engine.cpp", "api.cu", "rope_kernels.cu", "attn_fwd.cu", "score_kernel.cu", "topc_kernel.cu",
+           "rf_kernels.cu",
            "noalloc.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

@@ -20,7 +20,9 @@ def make_config(*, layers: int, heads: int, head_dim: int, grid_h: int, grid_w: 
                 policy: int = B.RC_SLIDING, mask_block_frames: int = 1, theta: float = 10000.0,
                 t_max: int = 4096, rope_pairs=(0, 0, 0), rs_bank_blocks: int = 0,
                 rs_sink_blocks: int = 0, rs_static_semantics: int = 0, ir_f_limit: int = 0,
-                ir_sink_blocks: int = 0, ir_cache_blocks: int = 0) -> B.rc_config:
+                ir_sink_blocks: int = 0, ir_cache_blocks: int = 0,
+                df_budget_tokens: int = 0, rf_history_frames: int = 0,
+                rf_weight: float = 0.5) -> B.rc_config:
     cfg = B.rc_config_init(layers, heads, head_dim, grid_h * grid_w, sink_frames, window_frames)
     cfg.grid_h, cfg.grid_w = grid_h, grid_w
     cfg.chunk_frames = chunk_frames
@@ -32,6 +34,8 @@ def make_config(*, layers: int, heads: int, head_dim: int, grid_h: int, grid_w: 
     cfg.rs_bank_blocks, cfg.rs_sink_blocks = rs_bank_blocks, rs_sink_blocks
     cfg.rs_static_semantics = rs_static_semantics
     cfg.ir_f_limit, cfg.ir_sink_blocks, cfg.ir_cache_blocks = ir_f_limit, ir_sink_blocks, ir_cache_blocks
+    cfg.df_budget_tokens = df_budget_tokens
+    cfg.rf_history_frames, cfg.rf_weight = rf_history_frames, rf_weight
     return cfg
 
 
@@ -112,6 +116,17 @@ class RollingKVCache:
             return out
         return out_dev
 
+    def comp_tokens(self, layer: int = 0):
+        """Deep Forcing: (frames, tokens) of the layer's compressed region, in
+        region order (synchronizes the cache's stream)."""
+        n = self.state(layer).comp_tokens
+        return B.rc_comp_tokens(self.handle, layer, n, self._stream())
+
+    def pool_scores(self, layer: int = 0):
+        """Relax Forcing: scores of the pool at the layer's last frame selection
+        (empty if its last new chunk needed none)."""
+        return B.rc_pool_scores(self.handle, layer, self._stream())
+
     def select_topc(self, layer: int, scores, C: int, topc=None):
         """Top-C over ``scores`` ([n_candidates] fp32 on this device, e.g. the
         sum of the head shards' score vectors) in ``layer``'s candidate order
@@ -152,16 +167,24 @@ class RollingKVCache:
         return self.mem[base + offset: base + offset + nbytes]
 
     def cache_views(self, layer: int):
-        """(K, V) torch views [H, capacity, d] bf16 of one layer's ring buffers."""
+        """(K, V) [H, capacity, d] bf16 of one layer's ring buffers.
+
+        The buffers keep each head in 64-dim planes ([H][d/64][capacity][64]);
+        for d > 64 the returned tensors are copies in token-major order (index
+        [h, t, j] is dim j of token row t), for d = 64 views."""
         if self.mem is None:
             raise RuntimeError("host-only handle")
         lay = B.rc_cache_layout(self.handle)
         H, d = self.cfg.heads, self.cfg.head_dim
-        n = H * lay.capacity * d * 2
+        P, cap = d // 64, lay.capacity
+        n = H * cap * d * 2
         o = layer * lay.kv_layer_stride
-        k = self._region(lay.k_offset + o, n).view(torch.bfloat16).view(H, lay.capacity, d)
-        v = self._region(lay.v_offset + o, n).view(torch.bfloat16).view(H, lay.capacity, d)
-        return k, v
+
+        def logical(off):
+            planes = self._region(off, n).view(torch.bfloat16).view(H, P, cap, 64)
+            return planes.permute(0, 2, 1, 3).flatten(2) if P > 1 else planes.view(H, cap, 64)
+
+        return logical(lay.k_offset + o), logical(lay.v_offset + o)
 
     def raw_views(self, layer: int):
         """(raw K, raw V or None) views [H, raw_frames*F, d] of the pristine source."""

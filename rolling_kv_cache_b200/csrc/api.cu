@@ -13,6 +13,7 @@
 #include "../../include/rc.h"
 #include "engine.hpp"
 #include "kernels.cuh"
+#include "df_compact.cuh"
 
 namespace {
 
@@ -30,11 +31,19 @@ rc_status cuda_err(cudaError_t e, const char* what) {
 constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
+// Raw (unrotated) source buffers a policy keeps per layer: K and V for
+// Rolling Sink's bank, K for Infinity-RoPE's sink and for Deep Forcing.
+int raw_buffers(const rc_config& c) {
+  if (c.policy == RC_ROLLING_SINK) return 2;
+  return (c.policy == RC_INFINITY_ROPE || c.policy == RC_DEEP_FORCING) ? 1 : 0;
+}
+
 struct MemPlan {
   size_t kv_bytes, raw_bytes, q_bytes, lse_bytes, score_bytes, tab_t, tab_h, tab_w, status_bytes,
-      part_o_bytes, part_lse_bytes;
+      part_o_bytes, part_lse_bytes, df_meta_bytes, df_sel_bytes, rf_desc_bytes, rf_pool_bytes,
+      rf_cur_bytes;
   size_t off_kv, off_raw, off_q, off_lse, off_score_phys, off_score_logical, off_tab_t, off_tab_h,
-      off_tab_w, off_status, off_part_o, off_part_lse, total;
+      off_tab_w, off_status, off_part_o, off_part_lse, off_df, off_rf_cur, total;
   int pt, ph, pw, cap, raw_frames, q_stride;
 };
 
@@ -44,7 +53,9 @@ MemPlan plan_memory(const rc_config& c, int raw_frames) {
   m.ph = c.rope_h_pairs;
   m.pw = c.rope_w_pairs;
   if (m.pt == 0 && m.ph == 0 && m.pw == 0) rc::DefaultPairs(c.head_dim, &m.pt, &m.ph, &m.pw);
-  m.cap = (c.sink_frames + c.window_frames) * c.frame_seqlen;
+  // ring rows, then two selected-region buffers (Deep Forcing tokens, Relax Forcing frames)
+  const int region = c.df_budget_tokens + c.rf_history_frames * c.frame_seqlen;
+  m.cap = (c.sink_frames + c.window_frames) * c.frame_seqlen + 2 * region;
   m.raw_frames = raw_frames;
   m.q_stride = c.chunk_frames * c.frame_seqlen;
   const size_t row = (size_t)c.head_dim * 2;
@@ -60,7 +71,17 @@ MemPlan plan_memory(const rc_config& c, int raw_frames) {
   // stream-K partial rows of the attention: 2 slots per persistent CTA, 256 query rows each
   m.part_o_bytes = align_up((size_t)2 * rc::kMaxPersistentCtas * 256 * c.head_dim * 4);
   m.part_lse_bytes = align_up((size_t)2 * rc::kMaxPersistentCtas * 256 * 4);
-  const int nraw = c.policy == RC_ROLLING_SINK ? 2 : (c.policy == RC_INFINITY_ROPE ? 1 : 0);
+  // Deep / Relax Forcing per layer: (frame, token) of both region buffers' tokens, and the selection
+  m.df_meta_bytes = align_up((size_t)2 * region * 8);
+  m.df_sel_bytes = align_up((size_t)region * 4);
+  // Relax Forcing per layer: frame descriptors [ring + 2 K slots][H][d] fp32, pool scores;
+  // per step: the chunk's descriptors and their partial sums
+  const bool rf = c.policy == RC_RELAX_FORCING;
+  m.rf_desc_bytes = rf ? align_up((size_t)(c.sink_frames + c.window_frames + 2 * c.rf_history_frames) *
+                                  c.heads * c.head_dim * 4) : 0;
+  m.rf_pool_bytes = rf ? align_up((RC_MAX_SLOTS + 1) * 4) : 0;
+  m.rf_cur_bytes = rf ? align_up((size_t)(1 + 32) * c.chunk_frames * c.heads * c.head_dim * 4) : 0;
+  const int nraw = raw_buffers(c);
   size_t o = 0;
   m.off_kv = o;
   o += 2 * m.kv_bytes * c.layers;
@@ -86,6 +107,10 @@ MemPlan plan_memory(const rc_config& c, int raw_frames) {
   o += m.part_o_bytes;
   m.off_part_lse = o;
   o += m.part_lse_bytes;
+  m.off_df = o;
+  o += (m.df_meta_bytes + m.df_sel_bytes + m.rf_desc_bytes + m.rf_pool_bytes) * c.layers;
+  m.off_rf_cur = o;
+  o += m.rf_cur_bytes;
   m.total = o;
   return m;
 }
@@ -193,6 +218,13 @@ struct Cache {
   int sm_count = 148;
   // candidate frames (slot, logical position) of each layer's last step, for rc_select_topc
   std::vector<std::vector<std::pair<int, int>>> last_cand;
+  // Deep Forcing per layer: region token sources [2][budget] and the pool selection [budget]
+  std::vector<int2*> df_meta;
+  std::vector<int*> df_sel;
+  // Relax Forcing per layer: frame descriptors and the last pool scores ([RC_MAX_SLOTS] + count)
+  std::vector<float*> rf_desc;
+  std::vector<float*> rf_pool;
+  float* rf_cur = nullptr;  // the chunk's descriptors + partial sums (per step)
 };
 
 rc_status check_handle(const void* h) {
@@ -255,7 +287,7 @@ rc_status rc_cache_create(const rc_config* cfg, void* dev_mem, size_t bytes, voi
     c->mem = static_cast<uint8_t*>(dev_mem);
     uint8_t* b = c->mem;
     const int L = cfg->layers;
-    const int nraw = cfg->policy == RC_ROLLING_SINK ? 2 : (cfg->policy == RC_INFINITY_ROPE ? 1 : 0);
+    const int nraw = raw_buffers(*cfg);
     for (int l = 0; l < L; ++l) {
       c->kc.push_back(reinterpret_cast<uint16_t*>(b + m.off_kv + (2 * (size_t)l) * m.kv_bytes));
       c->vc.push_back(reinterpret_cast<uint16_t*>(b + m.off_kv + (2 * (size_t)l + 1) * m.kv_bytes));
@@ -263,6 +295,11 @@ rc_status rc_cache_create(const rc_config* cfg, void* dev_mem, size_t bytes, voi
                                   : nullptr);
       c->rawv.push_back(nraw == 2 ? reinterpret_cast<uint16_t*>(b + m.off_raw + (nraw * (size_t)l + 1) * m.raw_bytes)
                                   : nullptr);
+      uint8_t* df = b + m.off_df + (m.df_meta_bytes + m.df_sel_bytes + m.rf_desc_bytes + m.rf_pool_bytes) * l;
+      c->df_meta.push_back(reinterpret_cast<int2*>(df));
+      c->df_sel.push_back(reinterpret_cast<int*>(df + m.df_meta_bytes));
+      c->rf_desc.push_back(reinterpret_cast<float*>(df + m.df_meta_bytes + m.df_sel_bytes));
+      c->rf_pool.push_back(reinterpret_cast<float*>(df + m.df_meta_bytes + m.df_sel_bytes + m.rf_desc_bytes));
     }
     c->qrot = reinterpret_cast<uint16_t*>(b + m.off_q);
     c->lse_scratch = reinterpret_cast<float*>(b + m.off_lse);
@@ -271,6 +308,7 @@ rc_status rc_cache_create(const rc_config* cfg, void* dev_mem, size_t bytes, voi
     c->status = reinterpret_cast<int*>(b + m.off_status);
     c->part_o = reinterpret_cast<float*>(b + m.off_part_o);
     c->part_lse = reinterpret_cast<float*>(b + m.off_part_lse);
+    c->rf_cur = reinterpret_cast<float*>(b + m.off_rf_cur);
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) == cudaSuccess &&
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
@@ -289,8 +327,10 @@ rc_status rc_cache_create(const rc_config* cfg, void* dev_mem, size_t bytes, voi
     c->tm_k.resize(L);
     c->tm_v.resize(L);
     for (int l = 0; l < L; ++l) {
-      if (rc_status st = make_map(&c->tm_k[l], c->kc[l], cfg->head_dim, m.cap, cfg->heads, m.cap)) return st;
-      if (rc_status st = make_map(&c->tm_v[l], c->vc[l], cfg->head_dim, m.cap, cfg->heads, m.cap)) return st;
+      // K/V rings: [H][d/64][cap][64], mapped as H*d/64 planes of cap x 64
+      const int planes = cfg->heads * (cfg->head_dim / 64);
+      if (rc_status st = make_map(&c->tm_k[l], c->kc[l], 64, m.cap, planes, m.cap)) return st;
+      if (rc_status st = make_map(&c->tm_v[l], c->vc[l], 64, m.cap, planes, m.cap)) return st;
     }
     e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_err(e, "cache init");
@@ -341,6 +381,83 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
   const MemPlan& m = c->mp;
   const int F = cfg.frame_seqlen, H = cfg.heads, d = cfg.head_dim;
   const int Nq = n_frames * F;
+
+  // Relax Forcing: the chunk's frame descriptors, then (pool over K frames) the selection
+  const bool rf_policy = cfg.policy == RC_RELAX_FORCING;
+  if (rf_policy) {
+    rc::RfDescParams dp{};
+    dp.k = static_cast<const uint16_t*>(k_new);
+    dp.desc_cur = c->rf_cur;
+    dp.n_frames = n_frames;
+    dp.F = F;
+    dp.H = H;
+    dp.d = d;
+    Timed tm(c->prof, RC_KERNEL_COMPACT, s, 0.0, (double)n_frames * F * H * d * 2);
+    if (cudaError_t e = rc::launch_rf_desc(dp, s)) return cuda_err(e, "descriptor launch");
+  }
+  const int vslots_ring = cfg.sink_frames + cfg.window_frames;
+  const int region_frames = c->engine->df_budget() / F;  // K for Relax Forcing
+  if (rf_policy && !plan.repeat) {  // no pool scores unless this chunk selects
+    if (cudaError_t e = cudaMemsetAsync(c->rf_pool[layer] + RC_MAX_SLOTS, 0, 4, s)) return cuda_err(e, "memset");
+  }
+  if (rf_policy && plan.df.use_sel) {
+    const rc::DfCompact& df = plan.df;
+    rc::RfSelectParams sp{};
+    sp.desc = c->rf_desc[layer];
+    sp.desc_cur = c->rf_cur;
+    sp.n_pool = df.n_old / F + df.n_e;
+    for (int v = 0; v < df.n_old / F; ++v) sp.pool_vslot[v] = vslots_ring + df.src_buf * region_frames + v;
+    for (int e = 0; e < df.n_e; ++e) sp.pool_vslot[df.n_old / F + e] = df.e_slot[e];
+    sp.n_tail = df.n_tail_kept;
+    for (int t = 0; t < df.n_tail_kept; ++t) sp.tail_vslot[t] = df.tail_slot[t];
+    sp.n_cur = n_frames;
+    sp.K = region_frames;
+    sp.F = F;
+    sp.H = H;
+    sp.d = d;
+    sp.weight = (float)cfg.rf_weight;
+    sp.sel = c->df_sel[layer];
+    sp.pool_scores = c->rf_pool[layer];
+    sp.n_scored = reinterpret_cast<int*>(c->rf_pool[layer] + RC_MAX_SLOTS);
+    Timed tm(c->prof, RC_KERNEL_COMPACT, s, 0.0, 0.0);
+    if (cudaError_t e = rc::launch_rf_select(sp, s)) return cuda_err(e, "frame selection launch");
+  }
+
+  // K7: Deep / Relax Forcing region gather (before the append reuses the leaving frames' slots)
+  if (plan.df.active) {
+    const rc::DfCompact& df = plan.df;
+    rc::DfCompactParams cp{};
+    cp.kc = c->kc[layer];
+    cp.vc = c->vc[layer];
+    cp.raw_k = c->rawk[layer];
+    const int budget = c->engine->df_budget();
+    cp.meta_src = c->df_meta[layer] + (size_t)df.src_buf * budget;
+    cp.meta_dst = c->df_meta[layer] + (size_t)df.dst_buf * budget;
+    cp.sel = df.use_sel ? c->df_sel[layer] : nullptr;
+    cp.H = H;
+    cp.d = d;
+    cp.F = F;
+    cp.cap = m.cap;
+    cp.src_row0 = df.src_row0;
+    cp.dst_row0 = df.dst_row0;
+    cp.n_old = df.n_old;
+    cp.n_new = df.n_new;
+    cp.n_e = df.n_e;
+    for (int e = 0; e < df.n_e; ++e) {
+      cp.e_slot[e] = df.e_slot[e];
+      cp.e_frame[e] = df.e_frame[e];
+    }
+    cp.tau_new0 = df.tau_new0;
+    cp.keep_time = df.keep_time ? 1 : 0;
+    cp.desc = rf_policy ? c->rf_desc[layer] : nullptr;
+    cp.src_vslot0 = vslots_ring + df.src_buf * region_frames;
+    cp.dst_vslot0 = vslots_ring + df.dst_buf * region_frames;
+    cp.rt = c->rt;
+    // raw key read + rotated key, raw key and value written, value read: 5 rows of d bf16
+    // (a Relax Forcing frame move: key and value read and written, 4 rows)
+    Timed tm(c->prof, RC_KERNEL_COMPACT, s, 0.0, (df.keep_time ? 4.0 : 5.0) * df.n_new * H * d * 2);
+    if (cudaError_t e = rc::launch_df_compact(cp, s)) return cuda_err(e, "compact launch");
+  }
 
   // K2: re-rotation jobs (before the append; they touch other slots)
   for (size_t j0 = 0; j0 < plan.jobs.size(); j0 += rc::kMaxJobs) {
@@ -401,13 +518,21 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
     Timed tm(c->prof, RC_KERNEL_APPEND, s, 0.0, bytes);
     if (cudaError_t e = rc::launch_append(ap, s)) return cuda_err(e, "append launch");
   }
+  if (rf_policy) {  // the chunk's descriptors go with its frames' slots
+    const size_t fb = (size_t)H * d * 4;
+    for (int r = 0; r < n_frames; ++r)
+      if (cudaError_t e = cudaMemcpyAsync(c->rf_desc[layer] + (size_t)ap.slot[r] * H * d, c->rf_cur + (size_t)r * H * d,
+                                          fb, cudaMemcpyDeviceToDevice, s))
+        return cuda_err(e, "descriptor copy");
+  }
 
   // K4: attention
   if (c->tm_q_rows != Nq) {
     if (rc_status st = make_map(&c->tm_q, c->qrot, d, Nq, H, m.q_stride)) return st;
     c->tm_q_rows = Nq;
   }
-  const bool want_scores = scores || topc;
+  const bool df_policy = cfg.policy == RC_DEEP_FORCING;
+  const bool want_scores = scores || topc || df_policy;
   float* lse_buf = lse ? lse : (want_scores ? c->lse_scratch : nullptr);
   rc::AttnParams at;
   std::memset(&at, 0, sizeof(at));
@@ -518,9 +643,26 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
       tp.cand_slot[i] = plan.cand[i].slot;
       tp.cand_lpos[i] = plan.cand[i].lpos;
     }
-    {
+    if (scores || topc) {
       Timed tm(c->prof, RC_KERNEL_TOPC, s, 0.0, (double)plan.cand.size() * F * 4 * 2);
       if (cudaError_t e = rc::launch_topc(tp, s)) return cuda_err(e, "topc launch");
+    }
+    // Deep Forcing: the next new chunk's region, chosen now from this step's scores
+    if (df_policy && plan.df_select) {
+      rc::TopCParams sp2;
+      std::memset(&sp2, 0, sizeof(sp2));
+      sp2.score_phys = c->score_phys;
+      sp2.scores_out = c->score_logical;
+      sp2.topc = c->df_sel[layer];
+      sp2.C = c->engine->df_budget();
+      sp2.F = F;
+      sp2.n_cand_frames = (int)plan.df_pool.size();
+      for (size_t i = 0; i < plan.df_pool.size(); ++i) {
+        sp2.cand_slot[i] = plan.df_pool[i].slot;
+        sp2.cand_lpos[i] = plan.df_pool[i].lpos;
+      }
+      Timed tm(c->prof, RC_KERNEL_TOPC, s, 0.0, (double)plan.df_pool.size() * F * 4 * 2);
+      if (cudaError_t e = rc::launch_topc(sp2, s)) return cuda_err(e, "pool top-C launch");
     }
   }
   return RC_OK;
@@ -624,9 +766,55 @@ rc_status rc_get_state(const void* handle, int layer, rc_state* out) {
     out->kept[e] = rc_frame_state{k.content, k.tau, k.region, k.rank, L.kept_slot[e], k.tau + L.shift};
     if (k.region == rc::kHist) nc += c->cfg.frame_seqlen;
   }
-  out->n_candidates = nc;
+  out->n_candidates = nc + L.comp_n;
+  out->valid_tokens += L.comp_n;
+  out->comp_tokens = L.comp_n;
+  out->comp_tau0 = L.comp_tau0;
+  out->comp_row0 = (c->cfg.sink_frames + c->cfg.window_frames) * c->cfg.frame_seqlen +
+                   L.comp_buf * c->engine->df_budget();
   out->n_evicted = (int)L.evicted.size();
   for (size_t i = 0; i < L.evicted.size() && i < RC_MAX_SLOTS; ++i) out->evicted[i] = L.evicted[i];
+  return RC_OK;
+}
+
+rc_status rc_comp_tokens(void* handle, int layer, int32_t* frame, int32_t* tok, void* stream) {
+  if (rc_status st = check_handle(handle)) return st;
+  Cache* c = static_cast<Cache*>(handle);
+  if ((c->cfg.policy != RC_DEEP_FORCING && c->cfg.policy != RC_RELAX_FORCING) || !c->device)
+    return set_err(RC_EINVAL, "rc_comp_tokens needs a Deep or Relax Forcing device handle");
+  if (layer < 0 || layer >= c->cfg.layers) return set_err(RC_EINVAL, "layer out of range");
+  const rc::LayerState& L = c->engine->layer(layer);
+  if (L.comp_n == 0) return RC_OK;
+  if (!frame || !tok) return set_err(RC_EINVAL, "null output array");
+  std::vector<int2> meta(L.comp_n);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int2* src = c->df_meta[layer] + (size_t)L.comp_buf * c->engine->df_budget();
+  if (cudaError_t e = cudaMemcpyAsync(meta.data(), src, meta.size() * sizeof(int2), cudaMemcpyDeviceToHost, s))
+    return cuda_err(e, "region metadata copy");
+  if (cudaError_t e = cudaStreamSynchronize(s)) return cuda_err(e, "stream sync");
+  for (int i = 0; i < L.comp_n; ++i) {
+    frame[i] = meta[i].x;
+    tok[i] = meta[i].y;
+  }
+  return RC_OK;
+}
+
+rc_status rc_pool_scores(void* handle, int layer, float* scores, int32_t* n, void* stream) {
+  if (rc_status st = check_handle(handle)) return st;
+  Cache* c = static_cast<Cache*>(handle);
+  if (c->cfg.policy != RC_RELAX_FORCING || !c->device)
+    return set_err(RC_EINVAL, "rc_pool_scores needs a Relax Forcing device handle");
+  if (layer < 0 || layer >= c->cfg.layers) return set_err(RC_EINVAL, "layer out of range");
+  if (!scores || !n) return set_err(RC_EINVAL, "null output");
+  std::vector<float> buf(RC_MAX_SLOTS + 1);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaError_t e = cudaMemcpyAsync(buf.data(), c->rf_pool[layer], buf.size() * 4, cudaMemcpyDeviceToHost, s))
+    return cuda_err(e, "pool score copy");
+  if (cudaError_t e = cudaStreamSynchronize(s)) return cuda_err(e, "stream sync");
+  int cnt = 0;
+  std::memcpy(&cnt, &buf[RC_MAX_SLOTS], 4);
+  *n = cnt;
+  for (int i = 0; i < cnt && i < RC_MAX_SLOTS; ++i) scores[i] = buf[i];
   return RC_OK;
 }
 
@@ -650,7 +838,7 @@ rc_status rc_cache_layout(const void* handle, rc_layout* out) {
   if (!out) return set_err(RC_EINVAL, "null layout");
   const Cache* c = static_cast<const Cache*>(handle);
   const MemPlan& m = c->mp;
-  const int nraw = c->cfg.policy == RC_ROLLING_SINK ? 2 : (c->cfg.policy == RC_INFINITY_ROPE ? 1 : 0);
+  const int nraw = raw_buffers(c->cfg);
   std::memset(out, 0, sizeof(*out));
   out->kv_layer_stride = 2 * m.kv_bytes;
   out->k_offset = m.off_kv;

@@ -218,14 +218,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         if (g >= 2 && !ptx::mbar_wait(&bar_ke[st], free_par, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
         ptx::mbar_arrive_expect_tx(&bar_kf[st], L::kTile);
         for (int k = 0; k < L::kSub; ++k)
-          ptx::tma_load_3d(&p.tm_k, &bar_kf[st], base + L::kK + st * L::kTile + k * kSubTileBytes, 64 * k,
-                           t.tok, jb.h);
+          ptx::tma_load_3d(&p.tm_k, &bar_kf[st], base + L::kK + st * L::kTile + k * kSubTileBytes, 0,
+                           t.tok, jb.h * L::kSub + k);
         nk[st]++;
         if (g >= 2 && !ptx::mbar_wait(&bar_ve[st], free_par, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
         ptx::mbar_arrive_expect_tx(&bar_vf[st], L::kTile);
         for (int k = 0; k < L::kSub; ++k)
-          ptx::tma_load_3d(&p.tm_v, &bar_vf[st], base + L::kV + st * L::kTile + k * kSubTileBytes, 64 * k,
-                           t.tok, jb.h);
+          ptx::tma_load_3d(&p.tm_v, &bar_vf[st], base + L::kV + st * L::kTile + k * kSubTileBytes, 0,
+                           t.tok, jb.h * L::kSub + k);
         nv[st]++;
       }
     }

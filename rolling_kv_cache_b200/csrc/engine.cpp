@@ -13,6 +13,12 @@
 //   blocks shift back by the same amount, times below 0 clamp to 0; KV flush
 //   keeps the global sink and the last block; RoPE cut adds a jump to the
 //   time of everything after the switch point.
+// Deep Forcing -- rCM guide, strategy 4: deep sink + the top-C scored tokens
+//   + the recent tail; after compaction the sink's and the compressed
+//   region's time encodings are rewritten so no empty time positions remain
+//   (the readings are spelled out in include/rc.h, RC_DEEP_FORCING). The
+//   engine plans the region by counts and time formulas only; which tokens it
+//   holds is decided on the device from the scores.
 //
 // The ring buffer replaces the pages' left-shift of the cache: frame g of the
 // window lives in slot sink + (g - sink) mod window, so eviction is a table
@@ -49,7 +55,12 @@ rc_status ValidateConfig(const rc_config& c, std::string* err) {
     return Fail(err, "chunk_frames must be in [1, 16]");
   if (c.sink_frames < 0 || c.window_frames < 1) return Fail(err, "bad sink/window frames");
   if (c.sink_frames + c.window_frames > RC_MAX_SLOTS) return Fail(err, "sink + window exceeds 256 frames");
-  long long cap = (long long)(c.sink_frames + c.window_frames) * c.frame_seqlen;
+  if (c.df_budget_tokens != 0 && c.policy != RC_DEEP_FORCING)
+    return Fail(err, "df_budget_tokens is a Deep Forcing parameter");
+  if (c.rf_history_frames != 0 && c.policy != RC_RELAX_FORCING)
+    return Fail(err, "rf_history_frames is a Relax Forcing parameter");
+  long long cap = (long long)(c.sink_frames + c.window_frames) * c.frame_seqlen + 2LL * c.df_budget_tokens +
+                  2LL * c.rf_history_frames * c.frame_seqlen;
   if (cap * c.heads * c.head_dim >= (1LL << 31)) return Fail(err, "cache too large for 32-bit indexing");
   if ((long long)c.chunk_frames * c.frame_seqlen * c.heads * c.head_dim >= (1LL << 31))
     return Fail(err, "chunk too large for 32-bit indexing");
@@ -82,6 +93,22 @@ rc_status ValidateConfig(const rc_config& c, std::string* err) {
                          "(cache - sink + 1)*chunk frames");
       if (c.ir_f_limit < B) return Fail(err, "f_limit must be >= chunk_frames");
       break;
+    case RC_DEEP_FORCING:
+      if (c.window_frames < 2 * B) return Fail(err, "deep forcing needs a tail of at least two chunks");
+      if (c.df_budget_tokens < 0 || c.df_budget_tokens % c.frame_seqlen)
+        return Fail(err, "df_budget_tokens must be a non-negative multiple of frame_seqlen");
+      if (c.sink_frames + c.window_frames + c.df_budget_tokens / c.frame_seqlen > RC_MAX_SLOTS)
+        return Fail(err, "sink + tail + budget frames exceed 256");
+      break;
+    case RC_RELAX_FORCING:
+      if (c.window_frames < B) return Fail(err, "the tail must hold a whole chunk");
+      if (c.rf_history_frames < 0) return Fail(err, "rf_history_frames must be >= 0");
+      if (c.sink_frames + c.window_frames + c.rf_history_frames > RC_MAX_SLOTS)
+        return Fail(err, "sink + tail + history frames exceed 256");
+      if (!(c.rf_weight >= 0.0 && c.rf_weight <= 1.0)) return Fail(err, "rf_weight must be in [0, 1]");
+      if (c.rf_history_frames + B > 64) return Fail(err, "history frames + chunk frames must be <= 64");
+      if (c.heads * c.head_dim > 6144) return Fail(err, "relax forcing needs heads * head_dim <= 6144");
+      break;
     default:
       return Fail(err, "unknown policy");
   }
@@ -94,6 +121,9 @@ Engine::Engine(const rc_config& cfg) : cfg_(cfg) {
   W_f_ = cfg.window_frames;
   P_ = S_f_ + W_f_;
   F_ = cfg.frame_seqlen;
+  // tokens of one selected-region buffer (Deep Forcing budget, Relax Forcing history)
+  C_ = cfg.policy == RC_DEEP_FORCING ? cfg.df_budget_tokens
+       : cfg.policy == RC_RELAX_FORCING ? cfg.rf_history_frames * cfg.frame_seqlen : 0;
   layers_.resize(cfg.layers);
   for (auto& L : layers_) L.slots.assign(P_, Slot());
 }
@@ -101,6 +131,9 @@ Engine::Engine(const rc_config& cfg) : cfg_(cfg) {
 int Engine::pristine_frames() const {
   if (cfg_.policy == RC_ROLLING_SINK) return cfg_.rs_bank_blocks * B_;
   if (cfg_.policy == RC_INFINITY_ROPE) return S_f_;
+  // Deep Forcing: raw keys of every ring slot and both region buffers, indexed
+  // like the cache's rows, so sink and region keys are always rotated from raw
+  if (cfg_.policy == RC_DEEP_FORCING) return P_ + 2 * (C_ / F_);
   return 0;
 }
 
@@ -160,6 +193,21 @@ std::vector<Kept> Engine::KeptSet(const LayerState& L) const {
       for (int g = g0; g < end; ++g) out.push_back({g, tau(g), kCur, g - g0});
       break;
     }
+    case RC_RELAX_FORCING: {
+      // every frame at its own index; the history frames sit in the region
+      for (int g = 0; g < std::min(S_f_, g0); ++g) out.push_back({g, g, kSink, -1});
+      for (int g = TailStart(end); g < g0; ++g) out.push_back({g, g, kHist, -1});
+      for (int g = g0; g < end; ++g) out.push_back({g, g, kCur, g - g0});
+      break;
+    }
+    case RC_DEEP_FORCING: {
+      // sink right before the region, region right before the tail (no holes)
+      const int g_t = TailStart(end), V = L.comp_n / F_;
+      for (int j = 0; j < std::min(S_f_, g0); ++j) out.push_back({j, g_t - V - S_f_ + j, kSink, -1});
+      for (int g = g_t; g < g0; ++g) out.push_back({g, g, kHist, -1});
+      for (int g = g0; g < end; ++g) out.push_back({g, g, kCur, g - g0});
+      break;
+    }
   }
   return out;
 }
@@ -186,6 +234,7 @@ rc_status Engine::Step(int layer, int frame_start, int n_frames, StepPlan* plan,
   if (layer < 0 || layer >= (int)layers_.size()) return Fail(err, "layer out of range");
   if (n_frames < 1 || n_frames > B_) return Fail(err, "n_frames must be in [1, chunk_frames]");
   LayerState L = layers_[layer];  // work on a copy; commit on success
+  DfCompact df;
   const bool repeat = L.cur_start >= 0 && frame_start == L.cur_start;
   if (repeat) {
     if (n_frames != L.cur_n) return Fail(err, "a repeated pass must cover the same frames");
@@ -199,7 +248,8 @@ rc_status Engine::Step(int layer, int frame_start, int n_frames, StepPlan* plan,
       }
       return RC_ESTATE;
     }
-    if (cfg_.policy == RC_ROLLING_SINK || cfg_.policy == RC_INFINITY_ROPE) {
+    if (cfg_.policy == RC_ROLLING_SINK || cfg_.policy == RC_INFINITY_ROPE || cfg_.policy == RC_DEEP_FORCING ||
+        cfg_.policy == RC_RELAX_FORCING) {
       if (n_frames != B_ || frame_start % B_) return Fail(err, "block policies step whole blocks");
     }
     if (cfg_.policy == RC_NONE && frame_start + n_frames > P_) {
@@ -207,6 +257,43 @@ rc_status Engine::Step(int layer, int frame_start, int n_frames, StepPlan* plan,
       return RC_ERANGE;
     }
     for (int g = frame_start; g < frame_start + n_frames; ++g) L.vtime.push_back(g + L.cut_total);
+    if (cfg_.policy == RC_DEEP_FORCING || cfg_.policy == RC_RELAX_FORCING) {
+      // pool = region tokens + the tokens of the frames leaving the tail (Relax
+      // Forcing selects whole frames of it, Deep Forcing single tokens)
+      DfCompact& d = df;
+      const int new_end = frame_start + n_frames;
+      d.n_old = L.comp_n;
+      d.n_e = 0;
+      for (int g = TailStart(L.end); g < TailStart(new_end) && g < L.end; ++g) {
+        const int s = S_f_ + (g - S_f_) % W_f_;
+        if (!L.slots[s].valid || L.slots[s].content != g) {
+          if (err) *err = "internal: a leaving tail frame is not in its slot";
+          return RC_EINVAL;
+        }
+        d.e_slot[d.n_e] = s;
+        d.e_frame[d.n_e] = g;
+        d.e_sigma[d.n_e] = L.slots[s].sigma;
+        ++d.n_e;
+      }
+      const int pool = d.n_old + d.n_e * F_;
+      d.n_new = std::min(C_, pool);
+      d.use_sel = C_ > 0 && pool > C_;
+      d.active = d.n_new > 0;
+      d.src_buf = L.comp_buf;
+      d.dst_buf = d.active ? 1 - L.comp_buf : L.comp_buf;
+      d.src_row0 = P_ * F_ + d.src_buf * C_;
+      d.dst_row0 = P_ * F_ + d.dst_buf * C_;
+      d.tau_old0 = L.comp_tau0;
+      d.tau_new0 = cfg_.policy == RC_RELAX_FORCING ? -1 : TailStart(new_end) - d.n_new / F_;
+      d.keep_time = cfg_.policy == RC_RELAX_FORCING;
+      // the tail after this chunk (Relax Forcing's alignment target): ring slots
+      // of the frames that stay, then the chunk's own frames
+      d.n_tail_kept = 0;
+      for (int g = TailStart(new_end); g < frame_start; ++g) d.tail_slot[d.n_tail_kept++] = S_f_ + (g - S_f_) % W_f_;
+      L.comp_n = d.n_new;
+      L.comp_buf = d.dst_buf;
+      L.comp_tau0 = d.tau_new0;
+    }
     L.end = frame_start + n_frames;
     L.cur_start = frame_start;
     L.cur_n = n_frames;
@@ -236,6 +323,7 @@ rc_status Engine::Step(int layer, int frame_start, int n_frames, StepPlan* plan,
   }
 
   StepPlan p;
+  p.df = df;
   p.repeat = repeat;
   p.frame_start = frame_start;
   p.n_frames = n_frames;
@@ -245,12 +333,16 @@ rc_status Engine::Step(int layer, int frame_start, int n_frames, StepPlan* plan,
     const Slot& have = L.slots[kslot[e]];
     const Slot& w = want[kslot[e]];
     if (k.region == kCur) {
-      p.append[k.rank] = AppendFrame{kslot[e], w.sigma, k.content < npr ? k.content : -1};
+      const int raw = cfg_.policy == RC_DEEP_FORCING ? kslot[e] : (k.content < npr ? k.content : -1);
+      p.append[k.rank] = AppendFrame{kslot[e], w.sigma, raw};
       continue;
     }
     if (have.valid && have.content == w.content && have.sigma == w.sigma) continue;
     const bool same = have.valid && have.content == w.content;
-    if (k.content < npr && (same || pristine_has_v())) {
+    if (cfg_.policy == RC_DEEP_FORCING && same) {
+      // sink moved in time: rotate again from its raw keys (raw row = slot row)
+      p.jobs.push_back(Job{kslot[e], kRotCopy, kslot[e], w.sigma, 0, 0});
+    } else if (k.content < npr && (same || pristine_has_v())) {
       p.jobs.push_back(Job{kslot[e], kRotCopy, k.content, w.sigma, 0, same ? 0 : 1});
     } else if (same) {
       int delta = w.sigma - have.sigma;
@@ -276,8 +368,28 @@ rc_status Engine::Step(int layer, int frame_start, int n_frames, StepPlan* plan,
     p.segs.push_back(Segment{s * F_, (t - s) * F_, cls[s]});
     s = t;
   }
+  // Deep Forcing: the region (logically between the sink and the history
+  // frames) is one more always-visible run; its V = comp_n / F "frames" are
+  // candidates with virtual slots past the ring (slot * F = its first row)
+  const int V = L.comp_n / F_;
+  const int vslot0 = P_ + L.comp_buf * (C_ / std::max(1, F_));
+  int n_sink = 0;
+  for (const Kept& k : kept) n_sink += k.region == kSink;
+  if (L.comp_n > 0) {
+    p.segs.push_back(Segment{P_ * F_ + L.comp_buf * C_, L.comp_n, -1});
+    for (int v = 0; v < V; ++v) p.cand.push_back(CandFrame{vslot0 + v, n_sink + v});
+  }
   for (size_t e = 0; e < kept.size(); ++e)
-    if (kept[e].region == kHist) p.cand.push_back(CandFrame{kslot[e], (int)e});
+    if (kept[e].region == kHist) p.cand.push_back(CandFrame{kslot[e], (int)e + V});
+  if (cfg_.policy == RC_DEEP_FORCING) {
+    // the next new chunk's pool: region + the tail frames it will push out
+    const int end = L.cur_start + L.cur_n;
+    for (int v = 0; v < V; ++v) p.df_pool.push_back(CandFrame{vslot0 + v, v});
+    int k = 0;
+    for (int g = TailStart(end); g < TailStart(end + B_); ++g, ++k)
+      p.df_pool.push_back(CandFrame{S_f_ + (g - S_f_) % W_f_, V + k});
+    p.df_select = C_ > 0 && L.comp_n + k * F_ > C_;
+  }
   if ((int)p.segs.size() > kEngineMaxSegs) {
     if (err) *err = "cache holds more KV runs than one attention launch takes";
     return RC_ERANGE;

@@ -11,6 +11,7 @@
 // segment list. Eviction is a slot-table update; no bytes move.
 #pragma once
 
+#include <algorithm>
 #include <cstdint>
 #include <string>
 #include <vector>
@@ -65,6 +66,26 @@ struct CandFrame {
   int lpos;       // its position in the logical kept list
 };
 
+// Deep Forcing compaction of one new chunk: the new compressed region is
+// gathered from the pool (old region tokens, then the tokens of the frames
+// that left the tail) into the other region buffer, each key re-rotated from
+// its old time to its new one.
+struct DfCompact {
+  bool active = false;
+  int src_row0 = 0, dst_row0 = 0;  // first physical row of the old / new region buffer
+  int src_buf = 0, dst_buf = 0;
+  int n_old = 0, n_new = 0;        // region tokens before / after
+  int n_e = 0;                     // frames that left the tail
+  int e_slot[RC_MAX_CHUNK_FRAMES];
+  int e_frame[RC_MAX_CHUNK_FRAMES];
+  int e_sigma[RC_MAX_CHUNK_FRAMES];
+  bool use_sel = false;            // pool > budget: region = the device top-C selection
+  int tau_old0 = 0, tau_new0 = 0;  // region token i: tau = tau0 + i / F (Deep Forcing)
+  bool keep_time = false;          // Relax Forcing: tokens keep their frame's time, no rotation
+  int n_tail_kept = 0;             // Relax Forcing: tail frames that stay (ring slots)
+  int tail_slot[RC_MAX_SLOTS];
+};
+
 struct StepPlan {
   bool repeat = false;
   int frame_start = 0;
@@ -73,6 +94,10 @@ struct StepPlan {
   std::vector<Job> jobs;
   std::vector<Segment> segs;
   std::vector<CandFrame> cand;  // logical order
+  // Deep Forcing
+  DfCompact df;
+  std::vector<CandFrame> df_pool;  // next new chunk's pool (lpos = pool frame index)
+  bool df_select = false;          // that pool exceeds the budget: select top-C now
 };
 
 struct LayerState {
@@ -89,6 +114,10 @@ struct LayerState {
   std::vector<int> kept_slot;
   std::vector<int> evicted;
   int n_jobs = 0;
+  // Deep Forcing compressed region
+  int comp_n = 0;     // tokens
+  int comp_buf = 0;   // which of the two region buffers holds it
+  int comp_tau0 = 0;  // region token i has tau = comp_tau0 + i / F
 };
 
 class Engine {
@@ -102,6 +131,10 @@ class Engine {
 
   const LayerState& layer(int l) const { return layers_[l]; }
   int slots() const { return P_; }
+  // Tokens per head the device buffers hold: the ring plus, under Deep
+  // Forcing, two compressed-region buffers of df_budget_tokens each.
+  long long capacity_tokens() const { return (long long)P_ * F_ + 2LL * C_; }
+  int df_budget() const { return C_; }
   // Frames of the pristine (raw, unrotated) source a policy keeps: Rolling
   // Sink's bank of the first K blocks (K and V), Infinity-RoPE's sink (K).
   int pristine_frames() const;
@@ -112,8 +145,10 @@ class Engine {
   int SlotOf(const LayerState& L, const Kept& k) const;
   int ShiftOf(const LayerState& L) const;
 
+  int TailStart(int end) const { return std::max(S_f_, end - W_f_); }
+
   rc_config cfg_;
-  int B_, S_f_, W_f_, P_, F_;
+  int B_, S_f_, W_f_, P_, F_, C_;
   std::vector<LayerState> layers_;
 };
 

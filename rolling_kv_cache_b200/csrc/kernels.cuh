@@ -35,7 +35,7 @@ struct AppendParams {
   const uint16_t* k;
   const uint16_t* v;
   uint16_t* q_rot;     // [H][q_stride][d]
-  uint16_t* kc;        // [H][cap][d]
+  uint16_t* kc;        // [H][d/64][cap][64]: 64-dim planes (cache_off)
   uint16_t* vc;
   uint16_t* raw_k;     // pristine [H][raw_cap][d] or null
   uint16_t* raw_v;     // pristine V (Rolling Sink bank) or null
@@ -76,8 +76,8 @@ struct KvSegment {
 // K4: chunk attention (one CTA per 128-query tile and head).
 struct alignas(64) AttnParams {
   CUtensorMap tm_q;    // q_rot [H][Nq][d], box {64, 128, 1}, 128B swizzle
-  CUtensorMap tm_k;    // K cache [H][cap][d]
-  CUtensorMap tm_v;    // V cache [H][cap][d]
+  CUtensorMap tm_k;    // K cache [H][d/64][cap][64] as (64, cap, H*d/64), box {64, 128, 1}
+  CUtensorMap tm_v;    // V cache, same layout
   uint16_t* out;       // [Nq][H][d] bf16
   float* lse;          // [H][Nq] or null
   int* status;         // device status word

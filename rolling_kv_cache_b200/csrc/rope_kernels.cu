@@ -14,6 +14,7 @@
 // uses separately rounded products (no fused multiply-add) so that a CPU fp32
 // restatement reproduces it bit for bit.
 #include "kernels.cuh"
+#include "df_compact.cuh"
 
 #include <cuda_bf16.h>
 
@@ -46,6 +47,15 @@ __device__ __forceinline__ float2 rope_cs(const RopeTables& rt, int m, int t, in
   if (m < rt.ph) return __ldg(rt.h + (size_t)hr * rt.ph + m);
   m -= rt.ph;
   return __ldg(rt.w + (size_t)wc * rt.pw + m);
+}
+
+// Element offset of (head h, token row t, 16-byte chunk c8) in a ring
+// buffer. K and V keep each head in d/64 planes of 64 dims, [H][d/64][cap][64],
+// so the time pairs (the first 2 P_t < 64 dims) of consecutive tokens sit in
+// dense 128-byte rows of plane 0 and an in-place time rotation reads and
+// writes 96 of every 128 bytes instead of 96 of every 256.
+__device__ __forceinline__ size_t cache_off(int h, int planes, int cap, int t, int c8) {
+  return (((size_t)h * planes + (c8 >> 3)) * cap + t) * 64 + (c8 & 7) * 8;
 }
 
 // (x, y) -> (x c - y s, x s + y c), products rounded separately.
@@ -84,7 +94,7 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
       rot(fk[2 * j], fk[2 * j + 1], cs.x, cs.y);
     }
     const size_t qdst = ((size_t)h * p.q_stride + tok) * p.d + c8 * 8;
-    const size_t cdst = ((size_t)h * p.cap + (size_t)p.slot[r] * p.F + n_in) * p.d + c8 * 8;
+    const size_t cdst = cache_off(h, p.d / 64, p.cap, p.slot[r] * p.F + n_in, c8);
     *reinterpret_cast<uint4*>(p.q_rot + qdst) = pack8(fq);
     *reinterpret_cast<uint4*>(p.kc + cdst) = pack8(fk);
     *reinterpret_cast<uint4*>(p.vc + cdst) = uv;
@@ -118,7 +128,7 @@ __global__ void __launch_bounds__(256) rerotate_kernel(const __grid_constant__ R
       const int c8 = i - row * ct;
       const int h = row / p.F;
       const int n_in = row - h * p.F;
-      const size_t dst = ((size_t)h * p.cap + (size_t)jb.dst_slot * p.F + n_in) * p.d + c8 * 8;
+      const size_t dst = cache_off(h, p.d / 64, p.cap, jb.dst_slot * p.F + n_in, c8);
       float f[8];
       uint4 u = *reinterpret_cast<const uint4*>(p.kc + dst);
       unpack8(u, f);
@@ -138,7 +148,7 @@ __global__ void __launch_bounds__(256) rerotate_kernel(const __grid_constant__ R
   for (int row = blockIdx.x * blockDim.y + threadIdx.y; row < rows; row += gridDim.x * blockDim.y) {
     const int h = row / p.F;
     const int n_in = row - h * p.F;
-    const size_t dst = ((size_t)h * p.cap + (size_t)jb.dst_slot * p.F + n_in) * p.d + c8 * 8;
+    const size_t dst = cache_off(h, p.d / 64, p.cap, jb.dst_slot * p.F + n_in, c8);
     float f[8];
     {
       const int hr = n_in / p.rt.grid_w;
@@ -155,6 +165,64 @@ __global__ void __launch_bounds__(256) rerotate_kernel(const __grid_constant__ R
       if (jb.copy_v)
         *reinterpret_cast<uint4*>(p.vc + dst) = __ldg(reinterpret_cast<const uint4*>(p.raw_v + src));
     }
+  }
+}
+
+// K7 Deep Forcing compaction (rCM guide, strategy 4: keep the top-C scored
+// tokens, then rewrite their time encoding so no holes remain). One thread
+// per 16-byte chunk of a (head, new region token) row, rows head-major so a
+// warp writes consecutive rows of one head; sources are gathered.
+__global__ void __launch_bounds__(256) df_compact_kernel(const __grid_constant__ DfCompactParams p) {
+  const int c8 = threadIdx.x;
+  const int rows = p.H * p.n_new;
+  const int planes = p.d / 64;
+  for (int r = blockIdx.x * blockDim.y + threadIdx.y; r < rows; r += gridDim.x * blockDim.y) {
+    const int h = r / p.n_new;
+    const int i = r - h * p.n_new;
+    const int pi = p.sel ? __ldg(p.sel + i) : i;
+    int src_row;
+    int2 meta;
+    if (pi < p.n_old) {
+      src_row = p.src_row0 + pi;
+      meta = p.meta_src[pi];
+    } else {
+      const int q = pi - p.n_old;
+      const int e = q / p.F;
+      const int t = q - e * p.F;
+      src_row = p.e_slot[e] * p.F + t;
+      meta = make_int2(p.e_frame[e], t);
+    }
+    const int dst_row = p.dst_row0 + i;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.vc + cache_off(h, planes, p.cap, src_row, c8)));
+    if (p.keep_time) {
+      // Relax Forcing: the key already sits at its frame's time; move it and
+      // the frame's descriptor (by the thread rows of the frame's first token)
+      *reinterpret_cast<uint4*>(p.kc + cache_off(h, planes, p.cap, dst_row, c8)) =
+          *reinterpret_cast<const uint4*>(p.kc + cache_off(h, planes, p.cap, src_row, c8));
+      if (i % p.F == 0) {
+        const int src_vs = pi < p.n_old ? p.src_vslot0 + pi / p.F : p.e_slot[(pi - p.n_old) / p.F];
+        const float4* sd = reinterpret_cast<const float4*>(p.desc + ((size_t)src_vs * p.H + h) * p.d + c8 * 8);
+        float4* dd = reinterpret_cast<float4*>(p.desc + ((size_t)(p.dst_vslot0 + i / p.F) * p.H + h) * p.d + c8 * 8);
+        dd[0] = sd[0];
+        dd[1] = sd[1];
+      }
+    } else {
+      const int hr = meta.y / p.rt.grid_w;
+      const int wc = meta.y - hr * p.rt.grid_w;
+      const int tau = p.tau_new0 + i / p.F;
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p.raw_k + ((size_t)h * p.cap + src_row) * p.d + c8 * 8));
+      float f[8];
+      unpack8(raw, f);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float2 cs = rope_cs(p.rt, c8 * 4 + j, tau, hr, wc);
+        rot(f[2 * j], f[2 * j + 1], cs.x, cs.y);
+      }
+      *reinterpret_cast<uint4*>(p.kc + cache_off(h, planes, p.cap, dst_row, c8)) = pack8(f);
+      *reinterpret_cast<uint4*>(p.raw_k + ((size_t)h * p.cap + dst_row) * p.d + c8 * 8) = raw;
+    }
+    *reinterpret_cast<uint4*>(p.vc + cache_off(h, planes, p.cap, dst_row, c8)) = v;
+    if (h == 0 && c8 == 0) p.meta_dst[i] = meta;
   }
 }
 
@@ -191,6 +259,17 @@ cudaError_t launch_rerotate(const RerotateParams& p, cudaStream_t s) {
   if (bx > cap) bx = cap;
   if (bx < 1) bx = 1;
   rerotate_kernel<<<dim3(bx, p.n_jobs), block, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_df_compact(const DfCompactParams& p, cudaStream_t s) {
+  const int rows = p.H * p.n_new;
+  if (rows == 0) return cudaSuccess;
+  const dim3 block(p.d / 8, 256 / (p.d / 8));
+  int blocks = (rows + block.y - 1) / block.y;
+  const int cap = sm_count() * 8;
+  if (blocks > cap) blocks = cap;
+  df_compact_kernel<<<blocks, block, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -179,8 +179,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const __grid_co
         }
         ptx::mbar_arrive_expect_tx(&bar_kf[st], L::kTile);
         for (int k = 0; k < L::kSub; ++k)
-          ptx::tma_load_3d(&p.tm_k, &bar_kf[st], base + L::kK + st * L::kTile + k * kSubTileBytes, 64 * k, t.tok,
-                           jb.h);
+          ptx::tma_load_3d(&p.tm_k, &bar_kf[st], base + L::kK + st * L::kTile + k * kSubTileBytes, 0, t.tok,
+                           jb.h * L::kSub + k);
         nk[st]++;
       }
     }

@@ -8,11 +8,11 @@ import numpy as np
 import torch
 
 import rc_synth
-from oracle import OracleStream
+from oracle import KeptToken, OracleStream
 from rolling_kv_cache_b200 import binding as B
 from rolling_kv_cache_b200.cache import RollingKVCache
 
-from rcutil import config_for, lib_kept, oracle_kept
+from rcutil import config_for, lib_kept, oracle_df_frames, oracle_kept
 
 TOL_MAX, TOL_MEAN, TOL_LSE = 2e-2, 2e-3, 1e-2
 
@@ -86,6 +86,9 @@ class Runner:
             self.pairs = rope_pair_split(w.head_dim)
         self.tables = [B.rc_rope_table(self.cache.handle, a) for a in range(3)]
         self.last = None
+        self.df = w.policy == rc_synth.POLICY_DEEP_FORCING
+        self.rf = w.policy == rc_synth.POLICY_RELAX_FORCING
+        self.prev_scores = None   # Deep Forcing: the last step's candidate scores (next pool)
 
     def step(self, chunk: int, pass_: int, cut: bool = False, scores: bool = False):
         w = self.w
@@ -96,16 +99,33 @@ class Runner:
         Nq = q.shape[0]
         lse = torch.empty((w.heads, Nq), dtype=torch.float32, device="cuda")
         sc = tc = None
-        if scores:
+        if scores or self.df:
             sc = torch.full((w.footprint_tokens,), -1.0, dtype=torch.float32, device="cuda")
+        if scores and w.topc:
             tc = torch.full((w.topc,), -7, dtype=torch.int32, device="cuda")
-        out = self.cache.step(self.layer, dev_bf16(q), dev_bf16(k), dev_bf16(v),
-                              chunk * w.chunk_frames, lse=lse, scores=sc, topc=tc, C=w.topc if scores else 0)
-        kept = self.oracle.step(chunk, pass_)
+        out = self.cache.step(self.layer, dev_bf16(q), dev_bf16(k), dev_bf16(v), chunk * w.chunk_frames,
+                              lse=lse, scores=sc, topc=tc, C=w.topc if tc is not None else 0)
+        if self.df:
+            # the region is chosen from the library's own scores of the last step (DF2)
+            kept = self.oracle.step(chunk, pass_, pool_scores=self.prev_scores)
+        else:
+            kept = self.oracle.step(chunk, pass_)
         torch.cuda.synchronize()
         self.cache.device_status()
         st = self.cache.state(self.layer)
-        assert lib_kept(st) == oracle_kept(kept)
+        if self.rf:
+            kept = self._check_rf_selection(st)
+        elif self.df:
+            assert lib_kept(st) == oracle_df_frames(kept)
+            comp = self.oracle.df.comp
+            assert st.comp_tokens == len(comp)
+            if comp:
+                frames, toks = self.cache.comp_tokens(self.layer)
+                assert list(zip(frames, toks)) == comp          # the selection, bit-exact
+                assert st.comp_tau0 == self.oracle.df.frame_taus()[1]
+            self.prev_scores = sc.cpu().numpy()[:st.n_candidates]
+        else:
+            assert lib_kept(st) == oracle_kept(kept)
         self.last = dict(q=q, k=k, v=v, out=bits_of(out), lse=lse.cpu().numpy(), state=st,
                          scores=None if sc is None else sc.cpu().numpy()[:st.n_candidates],
                          topc=None if tc is None else tc.cpu().numpy())
@@ -134,6 +154,66 @@ class Runner:
         want_q = rope_fp32(last["q"], tq, np.tile(hh, w.chunk_frames), np.tile(ww, w.chunk_frames),
                            self.tables, self.pairs)
         assert np.array_equal(qr, want_q)
+
+    def _check_rf_selection(self, st):
+        """Relax Forcing: the device's pool scores match fp64 within 1e-4, its
+        selection is the top-K of its own scores bit for bit, and differs from
+        the fp64 selection only among near-ties (then the oracle follows the
+        device's choice so both keep the same frames)."""
+        from oracle.relax_forcing import select_frames
+        rf, F = self.oracle.rf, self.w.frame_seqlen
+        gpu = np.array(self.cache.pool_scores(self.layer), dtype=np.float64)
+        if rf.last_scores is None:
+            assert len(gpu) == 0
+        else:
+            assert len(gpu) == len(rf.last_scores)
+            assert np.max(np.abs(gpu - rf.last_scores)) <= 1e-4, np.max(np.abs(gpu - rf.last_scores))
+            sel = select_frames(gpu.astype(np.float32), rf.K)
+            if sel != rf.last_selection:
+                kth = np.sort(rf.last_scores)[::-1][rf.K - 1]
+                for i in set(sel) ^ set(rf.last_selection):
+                    assert abs(rf.last_scores[i] - kth) <= 1e-4
+                rf.hist = [rf.last_pool[i] for i in sel]
+                rf.last_selection = sel
+        kept = rf.kept()
+        self.oracle.kept = kept
+        self.oracle.kept_tokens = [KeptToken(k.content, t, k.tau, k.region, k.rank) for k in kept for t in range(F)]
+        hist = set(rf.hist)
+        assert lib_kept(st) == [(k.content, k.tau, k.region, k.rank) for k in kept
+                                if not (k.region == "hist" and k.content in hist)]
+        assert st.comp_tokens == len(rf.hist) * F
+        if rf.hist:
+            frames, toks = self.cache.comp_tokens(self.layer)
+            assert frames == [g for g in rf.hist for _ in range(F)]
+            assert toks == list(range(F)) * len(rf.hist)
+        return kept
+
+    def check_df_region_bitexact(self):
+        """Deep Forcing: every region key == fp32 restatement of RoPE(raw key of
+        its source token) at the region's time for its position; V == raw v."""
+        w, st = self.w, self.last["state"]
+        if st.comp_tokens == 0:
+            return
+        F, Bf = w.frame_seqlen, w.chunk_frames
+        frames, toks = self.cache.comp_tokens(self.layer)
+        kc, vc = self.cache.cache_views(self.layer)
+        rows = slice(st.comp_row0, st.comp_row0 + st.comp_tokens)
+        got_k = bits_of(kc[:, rows]).transpose(1, 0, 2)
+        got_v = bits_of(vc[:, rows]).transpose(1, 0, 2)
+        raw_k = np.empty_like(got_k)
+        raw_v = np.empty_like(got_v)
+        frames, t = np.array(frames), np.array(toks)
+        for c in np.unique(frames // Bf):          # regenerate each source chunk once
+            kk, vv = (rc_synth.chunk_tensor(w, self.layer, int(c), self.oracle.last_pass[int(c)], tid, self.seed)
+                      for tid in (rc_synth.TENSOR_K, rc_synth.TENSOR_V))
+            sel = np.nonzero(frames // Bf == c)[0]
+            src = (frames[sel] % Bf) * F + t[sel]
+            raw_k[sel], raw_v[sel] = kk[src], vv[src]
+        # Deep Forcing: the region's packed times; Relax Forcing: each frame its own index
+        tau = frames if self.rf else st.comp_tau0 + np.arange(st.comp_tokens) // F
+        want_k = rope_fp32(raw_k, tau, t // w.grid_w, t % w.grid_w, self.tables, self.pairs)
+        assert np.array_equal(got_k, want_k)
+        assert np.array_equal(got_v, raw_v)
 
     def check_float(self, rows=None, heads=None, scores=False):
         ref = self.oracle.outputs(heads=heads, rows=rows, want_scores=scores)

@@ -13,7 +13,8 @@ def config_for(w: rc_synth.Workload, **over):
               theta=w.theta, t_max=w.t_max, rs_bank_blocks=w.rs_bank_blocks,
               rs_sink_blocks=w.rs_sink_blocks, rs_static_semantics=w.rs_static_semantics,
               ir_f_limit=w.ir_f_limit, ir_sink_blocks=w.ir_sink_blocks,
-              ir_cache_blocks=w.ir_cache_blocks)
+              ir_cache_blocks=w.ir_cache_blocks, df_budget_tokens=w.df_budget_tokens,
+              rf_history_frames=w.rf_history_frames, rf_weight=w.rf_weight)
     kw.update(over)
     return make_config(**kw)
 
@@ -24,3 +25,16 @@ def lib_kept(state):
 
 def oracle_kept(kept):
     return [(k.content, k.tau, k.region, k.rank) for k in kept]
+
+
+def oracle_df_frames(kept_tokens):
+    """Deep Forcing oracle tokens -> the frame entries the library reports
+    (sink, history, current; the compressed region is reported as a count)."""
+    out = []
+    for k in kept_tokens:
+        if k.region == "comp":
+            continue
+        e = (k.content, k.tau, k.region, k.rank)
+        if not out or out[-1] != e:
+            out.append(e)
+    return out

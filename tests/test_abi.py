@@ -25,10 +25,35 @@ def test_library_exports_every_declared_symbol():
     assert set(B.EXPORTS) <= set(names)
 
 
-def test_struct_sizes_match_header_layout():
-    # rc_config: 21 ints + 1 double, with the double 8-byte aligned
-    assert ctypes.sizeof(B.rc_frame_state) == 24
-    assert ctypes.sizeof(B.rc_state) == 4 * 8 + 4 * 256 + 4 + 24 * 256
+def _header_layout(structs):
+    """sizeof and offsetof of every field, as gcc lays the header's structs out."""
+    import shutil
+    import subprocess
+    import tempfile
+    if not shutil.which("gcc"):
+        pytest.skip("gcc not available")
+    lines = ['#include <stdio.h>', '#include "rc.h"', "int main(void) {"]
+    for st in structs:
+        name = st.__name__
+        lines.append(f'  printf("{name} %zu\\n", sizeof({name}));')
+        for f, _ in st._fields_:
+            lines.append(f'  printf("{name}.{f} %zu\\n", offsetof({name}, {f}));')
+    lines += ["  return 0;", "}"]
+    with tempfile.TemporaryDirectory() as d:
+        src, exe = os.path.join(d, "lay.c"), os.path.join(d, "lay")
+        open(src, "w").write("\n".join(lines))
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), src, "-o", exe], check=True)
+        out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout
+    return dict((k, int(v)) for k, v in (ln.split() for ln in out.splitlines()))
+
+
+def test_struct_layouts_match_header():
+    structs = [B.rc_config, B.rc_frame_state, B.rc_state, B.rc_layout, B.rc_profile]
+    lay = _header_layout(structs)
+    for st in structs:
+        assert ctypes.sizeof(st) == lay[st.__name__], st.__name__
+        for f, _ in st._fields_:
+            assert getattr(st, f).offset == lay[f"{st.__name__}.{f}"], (st.__name__, f)
 
 
 def test_config_init_and_bytes():

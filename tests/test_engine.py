@@ -13,10 +13,90 @@ from oracle import PolicyOracle
 from oracle.policy import evicted_contents
 from rolling_kv_cache_b200 import binding as B
 
-from rcutil import config_for, lib_kept, oracle_kept
+from rcutil import config_for, lib_kept, oracle_df_frames, oracle_kept
+
+
+def run_df_stream(w, seed=0):
+    """Deep Forcing: the engine plans the region by counts and times only
+    (which tokens it holds is decided on the device), so the oracle gets
+    arbitrary pool scores here and the frame list, region size and region
+    time must match."""
+    import numpy as np
+    from oracle import DeepForcingOracle
+    rng = np.random.default_rng(seed)
+    cfg = config_for(w, layers=1)
+    h = B.rc_cache_create(cfg, 0, 0)
+    df = DeepForcingOracle(w.chunk_frames, w.sink_frames, w.window_frames, w.df_budget_tokens,
+                           w.frame_seqlen)
+    F = w.frame_seqlen
+    n = 0
+    prev_sink_tau = None
+    try:
+        for c, p, g0, cut in rc_synth.stream_schedule(w):
+            B.rc_step(h, 0, 0, 0, 0, g0, w.chunk_frames, w.policy, 0)
+            pool = rng.random(df.next_pool_size(w.chunk_frames)) if p == 0 else None
+            kt = df.step(g0, w.chunk_frames, pool_scores=pool)
+            st = B.rc_get_state(h, 0)
+            frames = oracle_df_frames(kt)
+            assert lib_kept(st) == frames, (c, p)
+            sink_tau, tau0, V = df.frame_taus()
+            assert st.comp_tokens == len(df.comp) == V * F
+            if V:
+                assert st.comp_tau0 == tau0
+            assert st.valid_tokens == len(kt)
+            assert st.n_candidates == sum(1 for k in kt if k.region in ("comp", "hist"))
+            # keys carry their own time (no uniform shift); the sink moves only at new chunks
+            assert all(e.stored_time == e.tau for e in st.kept[:st.n_kept])
+            moved = (prev_sink_tau is not None and len(prev_sink_tau) == len(sink_tau)
+                     and sink_tau != prev_sink_tau)
+            if p > 0:
+                assert st.n_jobs == 0
+            elif moved:
+                assert st.n_jobs >= 1
+            prev_sink_tau = sink_tau
+            n += 1
+    finally:
+        B.rc_cache_destroy(h)
+    return n
+
+
+def run_rf_stream(w, seed=0):
+    """Relax Forcing: the engine plans the history region by counts only
+    (which frames it holds is decided on the device from the descriptors), so
+    the oracle gets arbitrary descriptors here; the sink / tail / chunk frames
+    and the history size must match."""
+    import numpy as np
+    from oracle.relax_forcing import RelaxForcingOracle
+    rng = np.random.default_rng(seed)
+    desc = {}
+    rf = RelaxForcingOracle(w.chunk_frames, w.sink_frames, w.window_frames, w.rf_history_frames,
+                            w.rf_weight, lambda g: desc.setdefault(g, rng.standard_normal(4)))
+    h = B.rc_cache_create(config_for(w, layers=1), 0, 0)
+    F = w.frame_seqlen
+    n = 0
+    try:
+        for c, p, g0, cut in rc_synth.stream_schedule(w):
+            B.rc_step(h, 0, 0, 0, 0, g0, w.chunk_frames, w.policy, 0)
+            kept = rf.step(g0, w.chunk_frames)
+            st = B.rc_get_state(h, 0)
+            hist = set(rf.hist)
+            frames = [(k.content, k.tau, k.region, k.rank) for k in kept
+                      if not (k.region == "hist" and k.content in hist)]
+            assert lib_kept(st) == frames, (c, p)
+            assert st.comp_tokens == len(rf.hist) * F
+            assert st.valid_tokens == len(kept) * F
+            assert st.n_jobs == 0      # nothing is re-rotated
+            n += 1
+    finally:
+        B.rc_cache_destroy(h)
+    return n
 
 
 def run_stream(w, steps=None):
+    if w.policy == rc_synth.POLICY_DEEP_FORCING:
+        return run_df_stream(w)
+    if w.policy == rc_synth.POLICY_RELAX_FORCING:
+        return run_rf_stream(w)
     cfg = config_for(w, layers=1)
     h = B.rc_cache_create(cfg, 0, 0)
     pol = PolicyOracle.from_workload(w)
@@ -138,7 +218,7 @@ def test_engine_fuzz_against_oracle():
     rng = random.Random(1234)
     for trial in range(60):
         B_ = rng.randint(1, 4)
-        pol_kind = rng.choice([0, 1, 2, 3])
+        pol_kind = rng.choice([0, 1, 2, 3, 4, 5])
         if pol_kind == 2:
             K = rng.randint(2, 7)
             S = rng.randint(1, K - 1)
@@ -154,6 +234,18 @@ def test_engine_fuzz_against_oracle():
                 chunk_frames=B_, ir_sink_blocks=Sb, ir_cache_blocks=Cb, sink_frames=Sb * B_,
                 window_frames=(Cb - Sb + 1) * B_, ir_f_limit=rng.randint(B_, 30),
                 chunks=rng.randint(1, 40), cut_chunks=cuts, cut_delta=rng.randint(0, 25))
+        elif pol_kind == 5:
+            w = rc_synth.WORKLOADS["tiny"].replace(
+                policy=rc_synth.POLICY_RELAX_FORCING, grid_h=2, grid_w=2, chunk_frames=B_,
+                sink_frames=rng.randint(0, 4), window_frames=rng.randint(B_, B_ + 6),
+                rf_history_frames=rng.randint(0, 8), chunks=rng.randint(1, 30), passes=rng.randint(1, 2))
+        elif pol_kind == 4:
+            F = 4
+            w = rc_synth.WORKLOADS["tiny"].replace(
+                policy=rc_synth.POLICY_DEEP_FORCING, grid_h=2, grid_w=2, chunk_frames=B_,
+                sink_frames=rng.randint(0, 4), window_frames=rng.randint(2 * B_, 2 * B_ + 6),
+                df_budget_tokens=F * rng.randint(0, 8), chunks=rng.randint(1, 30),
+                passes=rng.randint(1, 2))
         else:
             S_f = rng.randint(0, 5)
             W_f = rng.randint(B_, 20)

@@ -200,12 +200,92 @@ def test_inplace_rerotation_bitexact():
     r.cache.reindex(5, B.RC_REINDEX_SINK)
     r.oracle.reindex(4, 5)
     r.step(4, 0)
+    kc, _ = r.cache.cache_views(0)   # (a copy: the ring keeps 64-dim planes)
     after = bits_of(kc[:, 0:2 * F])
     want = rope_fp32_delta(before.transpose(1, 0, 2), 5, r.tables, r.pairs).transpose(1, 0, 2)
     assert np.array_equal(after, want)
     r.check_float()
     r.step(5, 0)
     r.check_float()
+    r.close()
+
+
+def test_deep_forcing_small():
+    """Deep Forcing (rCM guide, strategy 4) on a small stream, every step: the
+    region's tokens (chosen on the device from the kernel's own scores) equal
+    the host top-C of those same scores bit for bit, region keys equal a CPU
+    restatement of RoPE from their raw keys at the region's time, O / LSE
+    within the float bar of fp64 and scores within 1e-3 of fp64."""
+    w = W["deep_forcing"].replace(heads=2, grid_h=8, grid_w=8, chunks=14, df_budget_tokens=4 * 64)
+    r = Runner(w)
+    compacted = 0
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        r.step(c, p, scores=True)
+        r.check_append_bitexact()
+        r.check_df_region_bitexact()
+        ref, _ = r.check_float(scores=True)
+        sg, sr = r.last["scores"], ref["scores"]
+        assert len(sg) == len(sr)
+        if len(sr):
+            assert np.max(np.abs(sg - sr)) <= 1e-3 * max(1.0, np.max(np.abs(sr)))
+        compacted += r.oracle.df.last_selection is not None
+    assert compacted >= 8
+    r.close()
+
+
+def test_deep_forcing_repeat_passes_and_zero_budget():
+    # the selection of a chunk is made from the last pass before it
+    w = W["deep_forcing"].replace(heads=2, grid_h=4, grid_w=8, chunks=9, passes=2,
+                                  df_budget_tokens=2 * 32)
+    r = Runner(w)
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        r.step(c, p)
+        r.check_df_region_bitexact()
+        r.check_float()
+    r.close()
+    w0 = w.replace(df_budget_tokens=0, passes=1)
+    r = Runner(w0)
+    for c, p, g0, cut in rc_synth.stream_schedule(w0):
+        r.step(c, p)
+        assert r.last["state"].comp_tokens == 0
+        r.check_float()
+    r.close()
+
+
+def test_relax_forcing_small():
+    """Relax Forcing (rCM guide, strategy 5) on a small stream, every step:
+    device pool scores within 1e-4 of fp64, the device selection = top-K of
+    its own scores, region frames bit-exact copies of their keys at their own
+    times, O / LSE within the float bar."""
+    w = W["relax_forcing"].replace(heads=2, grid_h=8, grid_w=8, chunks=16, rf_history_frames=4)
+    r = Runner(w)
+    selected = 0
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        r.step(c, p)
+        r.check_append_bitexact()
+        r.check_df_region_bitexact()
+        r.check_float()
+        selected += r.oracle.rf.last_scores is not None
+    assert selected >= 8
+    r.close()
+
+
+@pytest.mark.parametrize("weight", [0.0, 1.0])
+def test_relax_forcing_weights_passes_zero_history(weight):
+    w = W["relax_forcing"].replace(heads=2, grid_h=4, grid_w=8, chunks=12, passes=2,
+                                   rf_history_frames=3, rf_weight=weight)
+    r = Runner(w)
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        r.step(c, p)
+        r.check_df_region_bitexact()
+        r.check_float()
+    r.close()
+    w0 = w.replace(rf_history_frames=0, passes=1)
+    r = Runner(w0)
+    for c, p, g0, cut in rc_synth.stream_schedule(w0):
+        r.step(c, p)
+        assert r.last["state"].comp_tokens == 0
+        r.check_float()
     r.close()
 
 
@@ -256,3 +336,43 @@ def test_full_rolling_sink_sampled():
 def test_full_infinity_rope_sampled():
     w = W["infinity_rope"].replace(cut_chunks=(9, 27, 60))
     _sampled(w, steps={0, 6, 7, 9, 10}, scores_at={7, 9, 10})
+
+
+def test_full_deep_forcing_sampled():
+    """Full-size Deep Forcing stream (12 heads, 1560-token frames, 3-frame
+    deep sink + 18720-token region + 6-frame tail): the region selection
+    exact every step, region keys bit-exact, sampled rows within the bar."""
+    w = W["deep_forcing"]
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([SAMPLE_ROWS, rng.integers(0, w.query_tokens, 20)]))
+    r = Runner(w)
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        if c > 9:
+            break
+        r.step(c, p)
+        if c in (0, 3, 4, 8, 9):
+            r.check_append_bitexact()
+            r.check_df_region_bitexact()
+            r.check_float(rows=rows)
+    st = r.last["state"]
+    assert st.comp_tokens == w.df_budget_tokens and st.valid_tokens == w.footprint_tokens
+    r.close()
+
+
+def test_full_relax_forcing_sampled():
+    """Full-size Relax Forcing stream (12 heads, 1560-token frames, sink 3 +
+    12 history frames + tail 6): selection checks every step, region frames
+    bit-exact and sampled rows within the bar at a few steps."""
+    w = W["relax_forcing"]
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([SAMPLE_ROWS, rng.integers(0, w.query_tokens, 20)]))
+    r = Runner(w)
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        if c > 9:
+            break
+        r.step(c, p)
+        if c in (0, 3, 8, 9):
+            r.check_append_bitexact()
+            r.check_df_region_bitexact()
+            r.check_float(rows=rows)
+    r.close()

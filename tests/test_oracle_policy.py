@@ -49,9 +49,15 @@ def test_lingbot_worked_numbers():
                                w.window_frames, w.chunk_frames, w.chunks)
 
 
-@pytest.mark.parametrize("name", list(rc_synth.WORKLOADS))
+FRAME_POLICIES = [n for n, w in rc_synth.WORKLOADS.items()
+                  if w.policy not in (rc_synth.POLICY_DEEP_FORCING, rc_synth.POLICY_RELAX_FORCING)]
+
+
+@pytest.mark.parametrize("name", FRAME_POLICIES)
 def test_footprint_constant(name):
-    """valid tokens = min(history, footprint) every step; never more."""
+    """valid tokens = min(history, footprint) every step; never more.
+    (Deep / Relax Forcing footprints are pinned in test_oracle_deep_forcing.py /
+    test_oracle_relax_forcing.py.)"""
     w = rc_synth.WORKLOADS[name]
     pol = PolicyOracle.from_workload(w)
     P = w.footprint_frames
