@@ -157,3 +157,45 @@ def test_two_gloo_ranks_compute_identical_integer_state():
     res = sorted(out_q.get(timeout=10) for _ in range(2))
     assert [r[1] for r in res] == [6, 6]
     assert all(r[2] for r in res) and all(r[3] == 32 for r in res)
+
+
+def _ulysses_main(rank, world, port, out_q):
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from rolling_kv_cache_b200.shard import head_ranges, heads_to_seq, seq_to_heads, token_ranges
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        ok = []
+        for N, H, d in [(12, 4, 3), (13, 5, 2), (7, 3, 4)]:      # uneven tokens and heads
+            g = torch.Generator().manual_seed(N * 100 + H)
+            x = torch.randn(N, H, d, generator=g)                  # the whole chunk, same on every rank
+            t0, t1 = token_ranges(N, world)[rank]
+            h0, h1 = head_ranges(H, world)[rank]
+            xh = seq_to_heads(x[t0:t1].clone(), H)
+            ok.append(torch.equal(xh, x[:, h0:h1]))
+            back = heads_to_seq(xh * 2.0, H, t1 - t0)               # a per-head op, then back
+            ok.append(torch.equal(back, 2.0 * x[t0:t1]))
+        out_q.put((rank, ok))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_ulysses_swaps_round_trip(world):
+    """seq_to_heads gives each rank every token of its head range; heads_to_seq
+    returns a per-head result to the token owners (uneven splits included)."""
+    ctx = mp.get_context("spawn")
+    out_q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ulysses_main, args=(r, world, port, out_q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = [out_q.get(timeout=10) for _ in range(world)]
+    assert all(all(ok) for _, ok in res)
