@@ -16,6 +16,7 @@ from typing import List, Optional
 POLICY_NONE, POLICY_SLIDING, POLICY_ROLLING_SINK, POLICY_INFINITY_ROPE = 0, 1, 2, 3
 POLICY_DEEP_FORCING = 4   # token-level; see deep_forcing.py
 POLICY_RELAX_FORCING = 5  # frame selection by similarity; see relax_forcing.py
+POLICY_MEMROPE = 6        # EMA memory frames; see memrope.py
 
 REINDEX_FLUSH = 1   # keep the sink and the last block, drop the middle
 REINDEX_CUT = 2     # add t_delta to the virtual time of every later frame

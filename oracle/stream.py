@@ -15,9 +15,10 @@ from typing import Dict, List, Optional, Sequence
 import numpy as np
 
 import rc_synth
-from .policy import POLICY_DEEP_FORCING, POLICY_RELAX_FORCING, KeptFrame, PolicyOracle
+from .policy import POLICY_DEEP_FORCING, POLICY_MEMROPE, POLICY_RELAX_FORCING, KeptFrame, PolicyOracle
 from .deep_forcing import DeepForcingOracle, KeptToken
 from .relax_forcing import RelaxForcingOracle, frame_descriptor
+from .memrope import MemRopeOracle
 from .rope import rope_angles, rope_apply, token_grid_positions
 from .attention import column_scores, masked_sdpa, top_c, visibility
 
@@ -30,8 +31,12 @@ class OracleStream:
         self.w = w
         self.layer = layer
         self.seed = seed
-        self.df = self.rf = None
-        if w.policy == POLICY_DEEP_FORCING:
+        self.df = self.rf = self.mr = None
+        if w.policy == POLICY_MEMROPE:
+            self.policy = None
+            self.mr = MemRopeOracle(w.chunk_frames, w.sink_frames, w.window_frames, w.mr_alpha_long,
+                                    w.mr_alpha_short, w.frame_seqlen, self.frame_raw)
+        elif w.policy == POLICY_DEEP_FORCING:
             self.policy = None
             self.df = DeepForcingOracle(w.chunk_frames, w.sink_frames, w.window_frames,
                                         w.df_budget_tokens, w.frame_seqlen)
@@ -62,7 +67,10 @@ class OracleStream:
         B = self.w.chunk_frames
         # this pass's raw values are what the cache holds from now on (D1)
         self.last_pass[chunk] = pass_
-        if self.df is not None:
+        if self.mr is not None:
+            self.kept_tokens = self.mr.step(chunk * B, B)
+            self.kept = []
+        elif self.df is not None:
             self.kept_tokens = self.df.step(chunk * B, B, pool_scores, selection)
             self.kept = []
         elif self.rf is not None:
@@ -76,7 +84,7 @@ class OracleStream:
             self.kept_tokens = [KeptToken(k.content, t, k.tau, k.region, k.rank)
                                 for k in self.kept for t in range(F)]
         self.cur = (chunk, pass_)
-        return self.kept_tokens if self.df is not None else self.kept
+        return self.kept_tokens if (self.df is not None or self.mr is not None) else self.kept
 
     # ------------------------------------------------------------ inputs
     def tensor(self, chunk: int, pass_: int, tid: int) -> np.ndarray:
@@ -118,7 +126,8 @@ class OracleStream:
             while j + 1 < len(kt) and kt[j + 1].content == kt[i].content and kt[j + 1].region == kt[i].region:
                 j += 1
             toks = np.array([k.tok for k in kt[i:j + 1]])
-            out.append(self.frame_raw(kt[i].content, tid)[toks])
+            src = self.mr.memory(kt[i].content, tid) if kt[i].content < 0 else self.frame_raw(kt[i].content, tid)
+            out.append(src[toks])
             i = j + 1
         return np.concatenate(out)
 

@@ -26,6 +26,7 @@ TENSOR_Q, TENSOR_K, TENSOR_V = 0, 1, 2
 POLICY_NONE, POLICY_SLIDING, POLICY_ROLLING_SINK, POLICY_INFINITY_ROPE = 0, 1, 2, 3
 POLICY_DEEP_FORCING = 4
 POLICY_RELAX_FORCING = 5
+POLICY_MEMROPE = 6
 
 
 @dataclasses.dataclass(frozen=True)
@@ -63,6 +64,9 @@ class Workload:
     # Relax Forcing: history frames kept between sink and tail, alignment weight
     rf_history_frames: int = 0
     rf_weight: float = 0.5
+    # MemRoPE: EMA factors of the long- and short-term memory frames
+    mr_alpha_long: float = 0.0
+    mr_alpha_short: float = 0.0
     mask_block_frames: int = 1
     theta: float = 10000.0
     t_max: int = 4096
@@ -81,7 +85,8 @@ class Workload:
 
     @property
     def footprint_tokens(self) -> int:
-        return (self.footprint_frames + self.rf_history_frames) * self.frame_seqlen + self.df_budget_tokens
+        mem = 2 if self.policy == POLICY_MEMROPE else 0
+        return (self.footprint_frames + self.rf_history_frames + mem) * self.frame_seqlen + self.df_budget_tokens
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)

@@ -579,7 +579,7 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
   {
     // algorithmic FLOPs: 4 d H per visible (query, key) pair
     const rc::LayerState& Ls = c->engine->layer(layer);
-    double n_hist = 0;
+    double n_hist = Ls.comp_n;  // the Deep / Relax Forcing region, always visible
     for (const rc::Kept& k : Ls.kept) n_hist += k.region != rc::kCur ? F : 0;
     double pairs = 0;
     for (int r = 0; r < n_frames; ++r) {
