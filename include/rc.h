@@ -76,8 +76,10 @@ typedef enum rc_policy {
   RC_INFINITY_ROPE = 3,  /* Infinity-RoPE: block-relative time, clamp at 0, flush + cut */
   RC_DEEP_FORCING = 4,   /* Deep Forcing: deep sink + top-C scored tokens + recent tail
                             (rCM length-extrapolation guide, strategy 4); see below */
-  RC_RELAX_FORCING = 5   /* Relax Forcing: sink + K history frames chosen by cosine
+  RC_RELAX_FORCING = 5,  /* Relax Forcing: sink + K history frames chosen by cosine
                             similarity + recent tail (strategy 5); see below */
+  RC_MEMROPE = 6         /* MemRoPE: sink + long/short EMA memory frames of the evicted
+                            frames + window (strategy 5's MemRoPE tip); see below */
 } rc_policy;
 
 /* rc_reindex flags */
@@ -117,7 +119,21 @@ typedef struct rc_config {
                              tail including the current chunk (>= 2 chunks) */
   int rf_history_frames;  /* Relax Forcing: K, history frames kept between sink and tail */
   double rf_weight;       /* Relax Forcing: w in score = w * alignment + (1 - w) * complement */
+  double mr_alpha_long;   /* MemRoPE: EMA factor of the long-term memory frame */
+  double mr_alpha_short;  /* MemRoPE: EMA factor of the short-term memory frame */
 } rc_config;
+
+/* MemRoPE (rCM length-extrapolation guide, the MemRoPE tip under strategy 5):
+ * the cache is the sliding window (sink_frames + window_frames) plus two
+ * memory frames. Every frame that leaves the window, oldest first, is folded
+ * token by token into both memories, per head, for raw keys and values:
+ * M = a M + (1 - a) X with a = mr_alpha_long / mr_alpha_short (the first
+ * evicted frame initialises them), in fp32 on the device. Keys are kept raw and
+ * positioned for attention at every step: the long-term memory at time
+ * sink_frames (right after the sink), the short-term one at g_w - 1 (right
+ * before the first window frame g_w), each token at its own (h, w).
+ * rc_get_state lists them as history entries with content -1 (long) and -2
+ * (short). Chunks are whole blocks. */
 
 /* Relax Forcing (rCM length-extrapolation guide, strategy 5): the cache keeps
  * the sink (the first sink_frames frames), at most rf_history_frames history

@@ -133,6 +133,13 @@ WORKLOADS = {
         grid_h=30, grid_w=52, chunk_frames=3, sink_frames=3, window_frames=6,
         policy=POLICY_RELAX_FORCING, chunks=60, passes=1, dist="normal_frame_mean",
         rf_history_frames=12, rf_weight=0.5),
+    # MemRoPE (rCM page, MemRoPE tip): sink 3 + long/short EMA memory frames
+    # + window 16 frames; same 32760-token footprint.
+    "memrope": Workload(
+        name="memrope", workload_id=8, layers=1, heads=12, head_dim=128,
+        grid_h=30, grid_w=52, chunk_frames=3, sink_frames=3, window_frames=16,
+        policy=POLICY_MEMROPE, chunks=60, passes=1, dist="normal_frame_mean",
+        mr_alpha_long=0.9, mr_alpha_short=0.5),
 }
 
 

@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "librc.so")
 
 RC_OK, RC_EINVAL, RC_ESTATE, RC_ECUDA, RC_ERANGE, RC_ETIMEOUT, RC_ENOMEM = range(7)
-RC_NONE, RC_SLIDING, RC_ROLLING_SINK, RC_INFINITY_ROPE, RC_DEEP_FORCING, RC_RELAX_FORCING = range(6)
+RC_NONE, RC_SLIDING, RC_ROLLING_SINK, RC_INFINITY_ROPE, RC_DEEP_FORCING, RC_RELAX_FORCING, RC_MEMROPE = range(7)
 RC_REINDEX_FLUSH, RC_REINDEX_CUT, RC_REINDEX_SINK = 1, 2, 4
 RC_MAX_SLOTS = 256
 RC_MAX_CHUNK_FRAMES = 16
@@ -39,7 +39,8 @@ class rc_config(ctypes.Structure):
         ("rs_static_semantics", ctypes.c_int), ("ir_f_limit", ctypes.c_int),
         ("ir_sink_blocks", ctypes.c_int), ("ir_cache_blocks", ctypes.c_int),
         ("df_budget_tokens", ctypes.c_int), ("rf_history_frames", ctypes.c_int),
-        ("rf_weight", ctypes.c_double),
+        ("rf_weight", ctypes.c_double), ("mr_alpha_long", ctypes.c_double),
+        ("mr_alpha_short", ctypes.c_double),
     ]
 
 

@@ -22,7 +22,8 @@ def make_config(*, layers: int, heads: int, head_dim: int, grid_h: int, grid_w: 
                 rs_sink_blocks: int = 0, rs_static_semantics: int = 0, ir_f_limit: int = 0,
                 ir_sink_blocks: int = 0, ir_cache_blocks: int = 0,
                 df_budget_tokens: int = 0, rf_history_frames: int = 0,
-                rf_weight: float = 0.5) -> B.rc_config:
+                rf_weight: float = 0.5, mr_alpha_long: float = 0.0,
+                mr_alpha_short: float = 0.0) -> B.rc_config:
     cfg = B.rc_config_init(layers, heads, head_dim, grid_h * grid_w, sink_frames, window_frames)
     cfg.grid_h, cfg.grid_w = grid_h, grid_w
     cfg.chunk_frames = chunk_frames
@@ -36,6 +37,7 @@ def make_config(*, layers: int, heads: int, head_dim: int, grid_h: int, grid_w: 
     cfg.ir_f_limit, cfg.ir_sink_blocks, cfg.ir_cache_blocks = ir_f_limit, ir_sink_blocks, ir_cache_blocks
     cfg.df_budget_tokens = df_budget_tokens
     cfg.rf_history_frames, cfg.rf_weight = rf_history_frames, rf_weight
+    cfg.mr_alpha_long, cfg.mr_alpha_short = mr_alpha_long, mr_alpha_short
     return cfg
 
 

@@ -35,13 +35,13 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // Rolling Sink's bank, K for Infinity-RoPE's sink and for Deep Forcing.
 int raw_buffers(const rc_config& c) {
   if (c.policy == RC_ROLLING_SINK) return 2;
-  return (c.policy == RC_INFINITY_ROPE || c.policy == RC_DEEP_FORCING) ? 1 : 0;
+  return (c.policy == RC_INFINITY_ROPE || c.policy == RC_DEEP_FORCING || c.policy == RC_MEMROPE) ? 1 : 0;
 }
 
 struct MemPlan {
   size_t kv_bytes, raw_bytes, q_bytes, lse_bytes, score_bytes, tab_t, tab_h, tab_w, status_bytes,
       part_o_bytes, part_lse_bytes, df_meta_bytes, df_sel_bytes, rf_desc_bytes, rf_pool_bytes,
-      rf_cur_bytes;
+      rf_cur_bytes, mem_bytes;
   size_t off_kv, off_raw, off_q, off_lse, off_score_phys, off_score_logical, off_tab_t, off_tab_h,
       off_tab_w, off_status, off_part_o, off_part_lse, off_df, off_rf_cur, total;
   int pt, ph, pw, cap, raw_frames, q_stride;
@@ -55,7 +55,8 @@ MemPlan plan_memory(const rc_config& c, int raw_frames) {
   if (m.pt == 0 && m.ph == 0 && m.pw == 0) rc::DefaultPairs(c.head_dim, &m.pt, &m.ph, &m.pw);
   // ring rows, then two selected-region buffers (Deep Forcing tokens, Relax Forcing frames)
   const int region = c.df_budget_tokens + c.rf_history_frames * c.frame_seqlen;
-  m.cap = (c.sink_frames + c.window_frames) * c.frame_seqlen + 2 * region;
+  m.cap = (c.sink_frames + c.window_frames) * c.frame_seqlen + 2 * region +
+          (c.policy == RC_MEMROPE ? 2 * c.frame_seqlen : 0);  // MemRoPE: the two memory frames
   m.raw_frames = raw_frames;
   m.q_stride = c.chunk_frames * c.frame_seqlen;
   const size_t row = (size_t)c.head_dim * 2;
@@ -81,6 +82,8 @@ MemPlan plan_memory(const rc_config& c, int raw_frames) {
                                   c.heads * c.head_dim * 4) : 0;
   m.rf_pool_bytes = rf ? align_up((RC_MAX_SLOTS + 1) * 4) : 0;
   m.rf_cur_bytes = rf ? align_up((size_t)(1 + 32) * c.chunk_frames * c.heads * c.head_dim * 4) : 0;
+  // MemRoPE per layer: fp32 EMA state of keys and values of both memories
+  m.mem_bytes = c.policy == RC_MEMROPE ? align_up((size_t)4 * c.frame_seqlen * c.heads * c.head_dim * 4) : 0;
   const int nraw = raw_buffers(c);
   size_t o = 0;
   m.off_kv = o;
@@ -108,7 +111,7 @@ MemPlan plan_memory(const rc_config& c, int raw_frames) {
   m.off_part_lse = o;
   o += m.part_lse_bytes;
   m.off_df = o;
-  o += (m.df_meta_bytes + m.df_sel_bytes + m.rf_desc_bytes + m.rf_pool_bytes) * c.layers;
+  o += (m.df_meta_bytes + m.df_sel_bytes + m.rf_desc_bytes + m.rf_pool_bytes + m.mem_bytes) * c.layers;
   m.off_rf_cur = o;
   o += m.rf_cur_bytes;
   m.total = o;
@@ -225,6 +228,8 @@ struct Cache {
   std::vector<float*> rf_desc;
   std::vector<float*> rf_pool;
   float* rf_cur = nullptr;  // the chunk's descriptors + partial sums (per step)
+  // MemRoPE per layer: fp32 EMA state [2 (k, v)][2 (long, short)][F][H][d]
+  std::vector<float*> mem_state;
 };
 
 rc_status check_handle(const void* h) {
@@ -295,11 +300,14 @@ rc_status rc_cache_create(const rc_config* cfg, void* dev_mem, size_t bytes, voi
                                   : nullptr);
       c->rawv.push_back(nraw == 2 ? reinterpret_cast<uint16_t*>(b + m.off_raw + (nraw * (size_t)l + 1) * m.raw_bytes)
                                   : nullptr);
-      uint8_t* df = b + m.off_df + (m.df_meta_bytes + m.df_sel_bytes + m.rf_desc_bytes + m.rf_pool_bytes) * l;
+      uint8_t* df = b + m.off_df + (m.df_meta_bytes + m.df_sel_bytes + m.rf_desc_bytes + m.rf_pool_bytes +
+                                    m.mem_bytes) * l;
       c->df_meta.push_back(reinterpret_cast<int2*>(df));
       c->df_sel.push_back(reinterpret_cast<int*>(df + m.df_meta_bytes));
       c->rf_desc.push_back(reinterpret_cast<float*>(df + m.df_meta_bytes + m.df_sel_bytes));
       c->rf_pool.push_back(reinterpret_cast<float*>(df + m.df_meta_bytes + m.df_sel_bytes + m.rf_desc_bytes));
+      c->mem_state.push_back(reinterpret_cast<float*>(df + m.df_meta_bytes + m.df_sel_bytes + m.rf_desc_bytes +
+                                                      m.rf_pool_bytes));
     }
     c->qrot = reinterpret_cast<uint16_t*>(b + m.off_q);
     c->lse_scratch = reinterpret_cast<float*>(b + m.off_lse);
@@ -421,6 +429,37 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
     sp.n_scored = reinterpret_cast<int*>(c->rf_pool[layer] + RC_MAX_SLOTS);
     Timed tm(c->prof, RC_KERNEL_COMPACT, s, 0.0, 0.0);
     if (cudaError_t e = rc::launch_rf_select(sp, s)) return cuda_err(e, "frame selection launch");
+  }
+
+  // MemRoPE: fold the frames leaving the window into the memories (before the
+  // append reuses their slots) and place both memory frames at their times
+  if (plan.mem.active) {
+    const rc::MemUpdate& mu = plan.mem;
+    rc::MemUpdateParams up{};
+    up.kc = c->kc[layer];
+    up.vc = c->vc[layer];
+    up.raw_k = c->rawk[layer];
+    up.mem = c->mem_state[layer];
+    up.H = H;
+    up.d = d;
+    up.F = F;
+    up.cap = m.cap;
+    up.raw_cap = m.raw_frames * F;
+    up.n_e = mu.n_e;
+    for (int e = 0; e < mu.n_e; ++e) up.e_slot[e] = mu.e_slot[e];
+    up.initialised = mu.initialised ? 1 : 0;
+    up.a[0] = (float)cfg.mr_alpha_long;
+    up.b[0] = (float)(1.0 - cfg.mr_alpha_long);
+    up.a[1] = (float)cfg.mr_alpha_short;
+    up.b[1] = (float)(1.0 - cfg.mr_alpha_short);
+    up.tau[0] = mu.tau[0];
+    up.tau[1] = mu.tau[1];
+    up.row0 = (cfg.sink_frames + cfg.window_frames) * F;
+    up.rt = c->rt;
+    // per evicted frame: raw key + value read; state read + written; two memory rows written
+    const double bytes = (double)F * H * d * (mu.n_e * 2.0 * 2 + 2 * 2 * 4 * 2 + 2 * 2 * 2);
+    Timed tm(c->prof, RC_KERNEL_COMPACT, s, 0.0, bytes);
+    if (cudaError_t e = rc::launch_mem_update(up, s)) return cuda_err(e, "memory update launch");
   }
 
   // K7: Deep / Relax Forcing region gather (before the append reuses the leaving frames' slots)

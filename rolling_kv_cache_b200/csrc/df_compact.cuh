@@ -54,6 +54,25 @@ struct RfSelectParams {
   float* pool_scores;      // [RC_MAX_SLOTS]
   int* n_scored;           // pool size of this selection
 };
+// MemRoPE (rCM guide, MemRoPE tip): fold the frames leaving the window into
+// the long- and short-term EMA memories (fp32 state, raw keys and values)
+// and write both memory frames, keys rotated to their times, into the cache.
+struct MemUpdateParams {
+  uint16_t* kc;            // [H][d/64][cap][64]
+  uint16_t* vc;
+  const uint16_t* raw_k;   // [H][raw_cap][d] raw keys of the ring slots
+  float* mem;              // [2 (k, v)][2 (long, short)][F][H][d] fp32 state
+  int H, d, F, cap, raw_cap;
+  int n_e;                 // frames leaving the window, oldest first
+  int e_slot[RC_MAX_CHUNK_FRAMES];
+  int initialised;         // the state holds a folded frame already
+  float a[2], b[2];        // alpha, 1 - alpha of the long- and short-term memory
+  int tau[2];              // their times
+  int row0;                // cache row of memory token 0 (long), row0 + F (short)
+  RopeTables rt;
+};
+cudaError_t launch_mem_update(const MemUpdateParams& p, cudaStream_t s);
+
 cudaError_t launch_rf_desc(const RfDescParams& p, cudaStream_t s);
 cudaError_t launch_rf_select(const RfSelectParams& p, cudaStream_t s);
 

@@ -60,7 +60,7 @@ rc_status ValidateConfig(const rc_config& c, std::string* err) {
   if (c.rf_history_frames != 0 && c.policy != RC_RELAX_FORCING)
     return Fail(err, "rf_history_frames is a Relax Forcing parameter");
   long long cap = (long long)(c.sink_frames + c.window_frames) * c.frame_seqlen + 2LL * c.df_budget_tokens +
-                  2LL * c.rf_history_frames * c.frame_seqlen;
+                  2LL * c.rf_history_frames * c.frame_seqlen + (c.policy == RC_MEMROPE ? 2LL * c.frame_seqlen : 0);
   if (cap * c.heads * c.head_dim >= (1LL << 31)) return Fail(err, "cache too large for 32-bit indexing");
   if ((long long)c.chunk_frames * c.frame_seqlen * c.heads * c.head_dim >= (1LL << 31))
     return Fail(err, "chunk too large for 32-bit indexing");
@@ -100,6 +100,13 @@ rc_status ValidateConfig(const rc_config& c, std::string* err) {
       if (c.sink_frames + c.window_frames + c.df_budget_tokens / c.frame_seqlen > RC_MAX_SLOTS)
         return Fail(err, "sink + tail + budget frames exceed 256");
       break;
+    case RC_MEMROPE:
+      if (c.window_frames < B) return Fail(err, "window must hold a whole chunk");
+      if (c.sink_frames + c.window_frames + 2 > RC_MAX_SLOTS) return Fail(err, "sink + window + memory exceed 256");
+      if (!(c.mr_alpha_long >= 0.0 && c.mr_alpha_long <= 1.0 && c.mr_alpha_short >= 0.0 &&
+            c.mr_alpha_short <= 1.0))
+        return Fail(err, "mr_alpha_long / mr_alpha_short must be in [0, 1]");
+      break;
     case RC_RELAX_FORCING:
       if (c.window_frames < B) return Fail(err, "the tail must hold a whole chunk");
       if (c.rf_history_frames < 0) return Fail(err, "rf_history_frames must be >= 0");
@@ -134,6 +141,7 @@ int Engine::pristine_frames() const {
   // Deep Forcing: raw keys of every ring slot and both region buffers, indexed
   // like the cache's rows, so sink and region keys are always rotated from raw
   if (cfg_.policy == RC_DEEP_FORCING) return P_ + 2 * (C_ / F_);
+  if (cfg_.policy == RC_MEMROPE) return P_;  // raw keys of the ring, folded when a frame leaves
   return 0;
 }
 
@@ -193,6 +201,20 @@ std::vector<Kept> Engine::KeptSet(const LayerState& L) const {
       for (int g = g0; g < end; ++g) out.push_back({g, tau(g), kCur, g - g0});
       break;
     }
+    case RC_MEMROPE: {
+      // sliding window with the two memory frames (virtual slots P, P + 1) in
+      // place of the evicted frames: long term after the sink, short term
+      // right before the window
+      const int g_w = TailStart(end);
+      for (int g = 0; g < std::min(S_f_, g0); ++g) out.push_back({g, g, kSink, -1});
+      if (L.mem_folded) {
+        out.push_back({-1, S_f_, kHist, -1});
+        out.push_back({-2, g_w - 1, kHist, -1});
+      }
+      for (int g = g_w; g < g0; ++g) out.push_back({g, g, kHist, -1});
+      for (int g = g0; g < end; ++g) out.push_back({g, g, kCur, g - g0});
+      break;
+    }
     case RC_RELAX_FORCING: {
       // every frame at its own index; the history frames sit in the region
       for (int g = 0; g < std::min(S_f_, g0); ++g) out.push_back({g, g, kSink, -1});
@@ -235,6 +257,7 @@ rc_status Engine::Step(int layer, int frame_start, int n_frames, StepPlan* plan,
   if (n_frames < 1 || n_frames > B_) return Fail(err, "n_frames must be in [1, chunk_frames]");
   LayerState L = layers_[layer];  // work on a copy; commit on success
   DfCompact df;
+  MemUpdate mem;
   const bool repeat = L.cur_start >= 0 && frame_start == L.cur_start;
   if (repeat) {
     if (n_frames != L.cur_n) return Fail(err, "a repeated pass must cover the same frames");
@@ -249,7 +272,7 @@ rc_status Engine::Step(int layer, int frame_start, int n_frames, StepPlan* plan,
       return RC_ESTATE;
     }
     if (cfg_.policy == RC_ROLLING_SINK || cfg_.policy == RC_INFINITY_ROPE || cfg_.policy == RC_DEEP_FORCING ||
-        cfg_.policy == RC_RELAX_FORCING) {
+        cfg_.policy == RC_RELAX_FORCING || cfg_.policy == RC_MEMROPE) {
       if (n_frames != B_ || frame_start % B_) return Fail(err, "block policies step whole blocks");
     }
     if (cfg_.policy == RC_NONE && frame_start + n_frames > P_) {
@@ -294,6 +317,17 @@ rc_status Engine::Step(int layer, int frame_start, int n_frames, StepPlan* plan,
       L.comp_buf = d.dst_buf;
       L.comp_tau0 = d.tau_new0;
     }
+    if (cfg_.policy == RC_MEMROPE) {
+      MemUpdate& mu = mem;
+      const int new_end = frame_start + n_frames;
+      mu.initialised = L.mem_folded;
+      for (int g = TailStart(L.end); g < TailStart(new_end) && g < L.end; ++g)
+        mu.e_slot[mu.n_e++] = S_f_ + (g - S_f_) % W_f_;
+      if (mu.n_e > 0) L.mem_folded = true;
+      mu.active = L.mem_folded;
+      mu.tau[0] = S_f_;
+      mu.tau[1] = TailStart(new_end) - 1;
+    }
     L.end = frame_start + n_frames;
     L.cur_start = frame_start;
     L.cur_n = n_frames;
@@ -304,6 +338,14 @@ rc_status Engine::Step(int layer, int frame_start, int n_frames, StepPlan* plan,
   std::vector<int> kslot(kept.size());
   std::vector<Slot> want(P_);
   for (size_t e = 0; e < kept.size(); ++e) {
+    if (kept[e].content < 0) {  // a MemRoPE memory frame: rows past the ring, written by its own kernel
+      kslot[e] = P_ + (kept[e].content == -1 ? 0 : 1);
+      if (kept[e].tau < 0 || kept[e].tau >= cfg_.t_max) {
+        if (err) *err = "memory time index outside [0, t_max)";
+        return RC_ERANGE;
+      }
+      continue;
+    }
     int s = SlotOf(L, kept[e]);
     int sigma = kept[e].tau + shift;
     if (s < 0 || s >= P_ || want[s].valid) {
@@ -324,16 +366,19 @@ rc_status Engine::Step(int layer, int frame_start, int n_frames, StepPlan* plan,
 
   StepPlan p;
   p.df = df;
+  p.mem = mem;
   p.repeat = repeat;
   p.frame_start = frame_start;
   p.n_frames = n_frames;
   const int npr = pristine_frames();
   for (size_t e = 0; e < kept.size(); ++e) {
     const Kept& k = kept[e];
+    if (k.content < 0) continue;  // MemRoPE memory: updated by the memory kernel
     const Slot& have = L.slots[kslot[e]];
     const Slot& w = want[kslot[e]];
     if (k.region == kCur) {
-      const int raw = cfg_.policy == RC_DEEP_FORCING ? kslot[e] : (k.content < npr ? k.content : -1);
+      const int raw = (cfg_.policy == RC_DEEP_FORCING || cfg_.policy == RC_MEMROPE) ? kslot[e]
+                      : (k.content < npr ? k.content : -1);
       p.append[k.rank] = AppendFrame{kslot[e], w.sigma, raw};
       continue;
     }
@@ -360,7 +405,7 @@ rc_status Engine::Step(int layer, int frame_start, int n_frames, StepPlan* plan,
   // KV runs for the attention: maximal runs of valid slots with one mask class.
   std::vector<int> cls(P_, -2);
   for (size_t e = 0; e < kept.size(); ++e)
-    cls[kslot[e]] = kept[e].region == kCur ? kept[e].rank / cfg_.mask_block_frames : -1;
+    if (kslot[e] < P_) cls[kslot[e]] = kept[e].region == kCur ? kept[e].rank / cfg_.mask_block_frames : -1;
   for (int s = 0; s < P_;) {
     if (!want[s].valid) { ++s; continue; }
     int t = s + 1;
@@ -368,6 +413,7 @@ rc_status Engine::Step(int layer, int frame_start, int n_frames, StepPlan* plan,
     p.segs.push_back(Segment{s * F_, (t - s) * F_, cls[s]});
     s = t;
   }
+  if (L.mem_folded) p.segs.push_back(Segment{P_ * F_, 2 * F_, -1});  // the two MemRoPE memory frames
   // Deep Forcing: the region (logically between the sink and the history
   // frames) is one more always-visible run; its V = comp_n / F "frames" are
   // candidates with virtual slots past the ring (slot * F = its first row)

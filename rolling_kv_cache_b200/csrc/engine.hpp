@@ -86,6 +86,16 @@ struct DfCompact {
   int tail_slot[RC_MAX_SLOTS];
 };
 
+// MemRoPE memory update of one new chunk: fold the frames leaving the window
+// into the two EMA memories and rotate both to their positions.
+struct MemUpdate {
+  bool active = false;
+  bool initialised = false;        // a frame was folded before this chunk
+  int n_e = 0;                     // frames leaving the window, oldest first
+  int e_slot[RC_MAX_CHUNK_FRAMES];
+  int tau[2] = {0, 0};             // long-term, short-term memory time
+};
+
 struct StepPlan {
   bool repeat = false;
   int frame_start = 0;
@@ -98,6 +108,8 @@ struct StepPlan {
   DfCompact df;
   std::vector<CandFrame> df_pool;  // next new chunk's pool (lpos = pool frame index)
   bool df_select = false;          // that pool exceeds the budget: select top-C now
+  // MemRoPE
+  MemUpdate mem;
 };
 
 struct LayerState {
@@ -118,6 +130,8 @@ struct LayerState {
   int comp_n = 0;     // tokens
   int comp_buf = 0;   // which of the two region buffers holds it
   int comp_tau0 = 0;  // region token i has tau = comp_tau0 + i / F
+  // MemRoPE: a frame has been folded into the memories
+  bool mem_folded = false;
 };
 
 class Engine {
@@ -133,7 +147,8 @@ class Engine {
   int slots() const { return P_; }
   // Tokens per head the device buffers hold: the ring plus, under Deep
   // Forcing, two compressed-region buffers of df_budget_tokens each.
-  long long capacity_tokens() const { return (long long)P_ * F_ + 2LL * C_; }
+  long long capacity_tokens() const { return (long long)P_ * F_ + 2LL * C_ + (mem() ? 2LL * F_ : 0); }
+  bool mem() const { return cfg_.policy == RC_MEMROPE; }
   int df_budget() const { return C_; }
   // Frames of the pristine (raw, unrotated) source a policy keeps: Rolling
   // Sink's bank of the first K blocks (K and V), Infinity-RoPE's sink (K).

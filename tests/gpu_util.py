@@ -31,8 +31,13 @@ def f32(bits):
 
 def rope_fp32(x_bits, t_pos, h_pos, w_pos, tables, pairs):
     """The kernels' rotation restated in numpy fp32: x [n, H, d] bf16 bits."""
+    return rope_fp32_values(f32(x_bits).astype(np.float32), t_pos, h_pos, w_pos, tables, pairs)
+
+
+def rope_fp32_values(x, t_pos, h_pos, w_pos, tables, pairs):
+    """Same rotation of fp32 values x [n, H, d]; returns bf16 bits."""
     pt, ph, pw = pairs
-    x = f32(x_bits).astype(np.float32)
+    x = np.asarray(x, dtype=np.float32)
     n, H, d = x.shape
     c = np.empty((n, d // 2), np.float32)
     s = np.empty((n, d // 2), np.float32)
@@ -88,6 +93,9 @@ class Runner:
         self.last = None
         self.df = w.policy == rc_synth.POLICY_DEEP_FORCING
         self.rf = w.policy == rc_synth.POLICY_RELAX_FORCING
+        self.mr = w.policy == rc_synth.POLICY_MEMROPE
+        self.mem_state = None     # MemRoPE: fp32 restatement of the device EMA [2 kv][2 mem][F, H, d]
+        self.mem_folded = 0
         self.prev_scores = None   # Deep Forcing: the last step's candidate scores (next pool)
 
     def step(self, chunk: int, pass_: int, cut: bool = False, scores: bool = False):
@@ -115,6 +123,9 @@ class Runner:
         st = self.cache.state(self.layer)
         if self.rf:
             kept = self._check_rf_selection(st)
+        elif self.mr:
+            assert lib_kept(st) == oracle_df_frames(kept)
+            self._fold_memory()
         elif self.df:
             assert lib_kept(st) == oracle_df_frames(kept)
             comp = self.oracle.df.comp
@@ -187,6 +198,45 @@ class Runner:
             assert frames == [g for g in rf.hist for _ in range(F)]
             assert toks == list(range(F)) * len(rf.hist)
         return kept
+
+    def _fold_memory(self):
+        """MemRoPE: fold newly evicted frames into the fp32 restatement of the
+        device state, in the device's operation order."""
+        w, mr = self.w, self.oracle.mr
+        F, Bf = w.frame_seqlen, w.chunk_frames
+        a = [np.float32(w.mr_alpha_long), np.float32(w.mr_alpha_short)]
+        b = [np.float32(1.0 - w.mr_alpha_long), np.float32(1.0 - w.mr_alpha_short)]
+        for g in mr.folded[self.mem_folded:]:
+            c, o = divmod(g, Bf)
+            x = [f32(rc_synth.chunk_tensor(w, self.layer, c, self.oracle.last_pass[c], tid, self.seed)
+                     [o * F:(o + 1) * F]).astype(np.float32) for tid in (rc_synth.TENSOR_K, rc_synth.TENSOR_V)]
+            if self.mem_state is None:
+                self.mem_state = [[x[kv].copy(), x[kv].copy()] for kv in range(2)]
+            else:
+                for kv in range(2):
+                    for m in range(2):
+                        self.mem_state[kv][m] = ((a[m] * self.mem_state[kv][m]).astype(np.float32) +
+                                                 (b[m] * x[kv]).astype(np.float32)).astype(np.float32)
+        self.mem_folded = len(mr.folded)
+
+    def check_mem_bitexact(self):
+        """MemRoPE: both memory frames' K / V rows == the fp32 restatement,
+        keys rotated to the memories' times at each token's (h, w)."""
+        if self.mem_state is None:
+            return
+        w, st = self.w, self.last["state"]
+        F = w.frame_seqlen
+        kc, vc = self.cache.cache_views(self.layer)
+        t = np.arange(F)
+        mem = {e.content: e for e in st.kept[:st.n_kept] if e.content < 0}
+        for m, content in enumerate((-1, -2)):
+            e = mem[content]
+            rows = slice(e.slot * F, (e.slot + 1) * F)
+            want_k = rope_fp32_values(self.mem_state[0][m], np.full(F, e.tau), t // w.grid_w, t % w.grid_w,
+                                      self.tables, self.pairs)
+            assert np.array_equal(bits_of(kc[:, rows]).transpose(1, 0, 2), want_k), content
+            want_v = rc_synth.f32_to_bf16_bits(self.mem_state[1][m])
+            assert np.array_equal(bits_of(vc[:, rows]).transpose(1, 0, 2), want_v), content
 
     def check_df_region_bitexact(self):
         """Deep Forcing: every region key == fp32 restatement of RoPE(raw key of

@@ -14,7 +14,8 @@ def config_for(w: rc_synth.Workload, **over):
               rs_sink_blocks=w.rs_sink_blocks, rs_static_semantics=w.rs_static_semantics,
               ir_f_limit=w.ir_f_limit, ir_sink_blocks=w.ir_sink_blocks,
               ir_cache_blocks=w.ir_cache_blocks, df_budget_tokens=w.df_budget_tokens,
-              rf_history_frames=w.rf_history_frames, rf_weight=w.rf_weight)
+              rf_history_frames=w.rf_history_frames, rf_weight=w.rf_weight,
+              mr_alpha_long=w.mr_alpha_long, mr_alpha_short=w.mr_alpha_short)
     kw.update(over)
     return make_config(**kw)
 

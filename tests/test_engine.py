@@ -92,7 +92,36 @@ def run_rf_stream(w, seed=0):
     return n
 
 
+def run_mr_stream(w):
+    """MemRoPE: sliding window plus the two memory frames (content -1 long at
+    time S_f, -2 short right before the window) once a frame has left."""
+    import numpy as np
+    from oracle.memrope import MemRopeOracle
+    mr = MemRopeOracle(w.chunk_frames, w.sink_frames, w.window_frames, w.mr_alpha_long,
+                       w.mr_alpha_short, w.frame_seqlen, lambda g, tid: np.zeros((1, 1, 1)))
+    h = B.rc_cache_create(config_for(w, layers=1), 0, 0)
+    n = 0
+    try:
+        for c, p, g0, cut in rc_synth.stream_schedule(w):
+            B.rc_step(h, 0, 0, 0, 0, g0, w.chunk_frames, w.policy, 0)
+            kt = mr.step(g0, w.chunk_frames)
+            st = B.rc_get_state(h, 0)
+            assert lib_kept(st) == oracle_df_frames(kt), (c, p)
+            assert st.valid_tokens == len(kt)
+            P = w.sink_frames + w.window_frames
+            for e in st.kept[:st.n_kept]:
+                if e.content < 0:
+                    assert e.slot == P + (0 if e.content == -1 else 1)
+            assert st.n_jobs == 0
+            n += 1
+    finally:
+        B.rc_cache_destroy(h)
+    return n
+
+
 def run_stream(w, steps=None):
+    if w.policy == rc_synth.POLICY_MEMROPE:
+        return run_mr_stream(w)
     if w.policy == rc_synth.POLICY_DEEP_FORCING:
         return run_df_stream(w)
     if w.policy == rc_synth.POLICY_RELAX_FORCING:
@@ -218,7 +247,7 @@ def test_engine_fuzz_against_oracle():
     rng = random.Random(1234)
     for trial in range(60):
         B_ = rng.randint(1, 4)
-        pol_kind = rng.choice([0, 1, 2, 3, 4, 5])
+        pol_kind = rng.choice([0, 1, 2, 3, 4, 5, 6])
         if pol_kind == 2:
             K = rng.randint(2, 7)
             S = rng.randint(1, K - 1)
@@ -234,6 +263,11 @@ def test_engine_fuzz_against_oracle():
                 chunk_frames=B_, ir_sink_blocks=Sb, ir_cache_blocks=Cb, sink_frames=Sb * B_,
                 window_frames=(Cb - Sb + 1) * B_, ir_f_limit=rng.randint(B_, 30),
                 chunks=rng.randint(1, 40), cut_chunks=cuts, cut_delta=rng.randint(0, 25))
+        elif pol_kind == 6:
+            w = rc_synth.WORKLOADS["tiny"].replace(
+                policy=rc_synth.POLICY_MEMROPE, grid_h=2, grid_w=2, chunk_frames=B_,
+                sink_frames=rng.randint(0, 4), window_frames=rng.randint(B_, B_ + 6),
+                mr_alpha_long=0.9, mr_alpha_short=0.5, chunks=rng.randint(1, 30), passes=rng.randint(1, 2))
         elif pol_kind == 5:
             w = rc_synth.WORKLOADS["tiny"].replace(
                 policy=rc_synth.POLICY_RELAX_FORCING, grid_h=2, grid_w=2, chunk_frames=B_,

@@ -289,6 +289,24 @@ def test_relax_forcing_weights_passes_zero_history(weight):
     r.close()
 
 
+@pytest.mark.parametrize("alphas", [(0.9, 0.5), (0.0, 1.0)])
+def test_memrope_small(alphas):
+    """MemRoPE (rCM guide, MemRoPE tip) on a small stream, every step: memory
+    frames bit-exact against the fp32 restatement of the device EMA with keys
+    rotated to their times, O / LSE within the float bar of the fp64 oracle
+    (which folds in fp64)."""
+    w = W["memrope"].replace(heads=2, grid_h=8, grid_w=8, chunks=14, window_frames=6,
+                             mr_alpha_long=alphas[0], mr_alpha_short=alphas[1])
+    r = Runner(w)
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        r.step(c, p)
+        r.check_append_bitexact()
+        r.check_mem_bitexact()
+        r.check_float()
+    assert r.mem_folded >= 20
+    r.close()
+
+
 # ----------------------------------------------------------- full sizes
 SAMPLE_ROWS = np.array([0, 1, 127, 128, 1559, 1560, 1561, 3119, 3120, 4607, 4608, 4679])
 
@@ -374,5 +392,24 @@ def test_full_relax_forcing_sampled():
         if c in (0, 3, 8, 9):
             r.check_append_bitexact()
             r.check_df_region_bitexact()
+            r.check_float(rows=rows)
+    r.close()
+
+
+
+def test_full_memrope_sampled():
+    """Full-size MemRoPE stream (12 heads, 1560-token frames, sink 3 + 2 memory
+    frames + window 16): memory frames bit-exact every checked step."""
+    w = W["memrope"]
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([SAMPLE_ROWS, rng.integers(0, w.query_tokens, 20)]))
+    r = Runner(w)
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        if c > 9:
+            break
+        r.step(c, p)
+        if c in (0, 6, 7, 9):
+            r.check_append_bitexact()
+            r.check_mem_bitexact()
             r.check_float(rows=rows)
     r.close()

@@ -50,7 +50,8 @@ def test_lingbot_worked_numbers():
 
 
 FRAME_POLICIES = [n for n, w in rc_synth.WORKLOADS.items()
-                  if w.policy not in (rc_synth.POLICY_DEEP_FORCING, rc_synth.POLICY_RELAX_FORCING)]
+                  if w.policy not in (rc_synth.POLICY_DEEP_FORCING, rc_synth.POLICY_RELAX_FORCING,
+                                      rc_synth.POLICY_MEMROPE)]
 
 
 @pytest.mark.parametrize("name", FRAME_POLICIES)
