@@ -293,7 +293,8 @@ def run_ours(args, w):
                 layer_step(l, q, k, v, c * B_, out if out_buf is None else out_buf)
 
     chunk = 0
-    prefill = (w.footprint_frames + B_ - 1) // B_   # until the window is full
+    # until the cache is full (the Deep / Relax Forcing region and MemRoPE memory included)
+    prefill = (w.footprint_tokens // w.frame_seqlen + B_ - 1) // B_
     for _ in range(prefill):
         run_chunk(chunk)
         chunk += 1
