@@ -290,14 +290,30 @@ int sm_count() {
   return n;
 }
 
+// Blocks of 256 threads of `kernel` resident at once on the GPU. The
+// grid-stride kernels below launch at most one full wave: blocks beyond it
+// would only start when others finish their whole loops and leave the tail of
+// the launch to a few SMs.
+template <typename Kernel>
+int one_wave(Kernel kernel, int* cache) {
+  if (*cache == 0) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess || per_sm < 1)
+      per_sm = 4;
+    *cache = per_sm * sm_count();
+  }
+  return *cache;
+}
+
 }  // namespace
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
   const int rows = p.n_tok * p.H;
   if (rows == 0) return cudaSuccess;
   const dim3 block(p.d / 8, 256 / (p.d / 8));
+  static int wave = 0;
   int blocks = (rows + block.y - 1) / block.y;
-  const int cap = sm_count() * 8;  // 8 resident 256-thread blocks per SM
+  const int cap = one_wave(append_kernel, &wave);
   if (blocks > cap) blocks = cap;
   append_kernel<<<blocks, block, 0, s>>>(p);
   return cudaGetLastError();
@@ -308,7 +324,8 @@ cudaError_t launch_rerotate(const RerotateParams& p, cudaStream_t s) {
   const dim3 block(p.d / 8, 256 / (p.d / 8));
   const int rows = p.F * p.H;
   int bx = (rows + block.y - 1) / block.y;
-  const int cap = (sm_count() * 8 + p.n_jobs - 1) / p.n_jobs;
+  static int wave = 0;
+  const int cap = one_wave(rerotate_kernel, &wave) / p.n_jobs;
   if (bx > cap) bx = cap;
   if (bx < 1) bx = 1;
   rerotate_kernel<<<dim3(bx, p.n_jobs), block, 0, s>>>(p);
@@ -318,8 +335,9 @@ cudaError_t launch_rerotate(const RerotateParams& p, cudaStream_t s) {
 cudaError_t launch_mem_update(const MemUpdateParams& p, cudaStream_t s) {
   const int rows = p.F * p.H;
   const dim3 block(p.d / 8, 256 / (p.d / 8));
+  static int wave = 0;
   int blocks = (rows + block.y - 1) / block.y;
-  const int cap = sm_count() * 8;
+  const int cap = one_wave(mem_update_kernel, &wave);
   if (blocks > cap) blocks = cap;
   mem_update_kernel<<<blocks, block, 0, s>>>(p);
   return cudaGetLastError();
@@ -329,8 +347,9 @@ cudaError_t launch_df_compact(const DfCompactParams& p, cudaStream_t s) {
   const int rows = p.H * p.n_new;
   if (rows == 0) return cudaSuccess;
   const dim3 block(p.d / 8, 256 / (p.d / 8));
+  static int wave = 0;
   int blocks = (rows + block.y - 1) / block.y;
-  const int cap = sm_count() * 8;
+  const int cap = one_wave(df_compact_kernel, &wave);
   if (blocks > cap) blocks = cap;
   df_compact_kernel<<<blocks, block, 0, s>>>(p);
   return cudaGetLastError();
