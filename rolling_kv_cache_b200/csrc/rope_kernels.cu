@@ -226,56 +226,59 @@ __global__ void __launch_bounds__(256) df_compact_kernel(const __grid_constant__
   }
 }
 
-// MemRoPE update: one thread per 16-byte chunk of a (token, head) row of
-// the memory frames; the EMA runs in fp32 with separately rounded products so
-// a CPU fp32 restatement reproduces it bit for bit.
+// MemRoPE update: one thread per 16-byte chunk of a (memory, token, head)
+// row; the EMA runs in fp32 with separately rounded products so a CPU fp32
+// restatement reproduces it bit for bit.
 __global__ void __launch_bounds__(256) mem_update_kernel(const __grid_constant__ MemUpdateParams p) {
   const int c8 = threadIdx.x;
-  const int rows = p.F * p.H;
+  const int per_mem = p.F * p.H;
+  const int rows = 2 * per_mem;
   const int planes = p.d / 64;
   for (int r = blockIdx.x * blockDim.y + threadIdx.y; r < rows; r += gridDim.x * blockDim.y) {
-    const int t = r / p.H;
-    const int h = r - t * p.H;
+    const int m = r >= per_mem;          // 0 long-term, 1 short-term
+    const int rr = r - m * per_mem;
+    const int t = rr / p.H;
+    const int h = rr - t * p.H;
+    float* sk = p.mem + (((size_t)(0 * 2 + m) * p.F + t) * p.H + h) * p.d + c8 * 8;
+    float* sv = p.mem + (((size_t)(1 * 2 + m) * p.F + t) * p.H + h) * p.d + c8 * 8;
+    float k[8], v[8];
+    if (p.initialised) {
+      const float4* k4 = reinterpret_cast<const float4*>(sk);
+      const float4* v4 = reinterpret_cast<const float4*>(sv);
+      const float4 k0 = k4[0], k1 = k4[1], v0 = v4[0], v1 = v4[1];
+      k[0] = k0.x; k[1] = k0.y; k[2] = k0.z; k[3] = k0.w; k[4] = k1.x; k[5] = k1.y; k[6] = k1.z; k[7] = k1.w;
+      v[0] = v0.x; v[1] = v0.y; v[2] = v0.z; v[3] = v0.w; v[4] = v1.x; v[5] = v1.y; v[6] = v1.z; v[7] = v1.w;
+    }
+    for (int e = 0; e < p.n_e; ++e) {
+      const int row = p.e_slot[e] * p.F + t;
+      float xk[8], xv[8];
+      unpack8(__ldg(reinterpret_cast<const uint4*>(p.raw_k + ((size_t)h * p.raw_cap + row) * p.d + c8 * 8)), xk);
+      unpack8(__ldg(reinterpret_cast<const uint4*>(p.vc + cache_off(h, planes, p.cap, row, c8))), xv);
+      const bool first = !p.initialised && e == 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        k[j] = first ? xk[j] : __fadd_rn(__fmul_rn(p.a[m], k[j]), __fmul_rn(p.b[m], xk[j]));
+        v[j] = first ? xv[j] : __fadd_rn(__fmul_rn(p.a[m], v[j]), __fmul_rn(p.b[m], xv[j]));
+      }
+    }
+    if (p.n_e > 0) {
+      float4* k4 = reinterpret_cast<float4*>(sk);
+      float4* v4 = reinterpret_cast<float4*>(sv);
+      k4[0] = make_float4(k[0], k[1], k[2], k[3]);
+      k4[1] = make_float4(k[4], k[5], k[6], k[7]);
+      v4[0] = make_float4(v[0], v[1], v[2], v[3]);
+      v4[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
     const int hr = t / p.rt.grid_w;
     const int wc = t - hr * p.rt.grid_w;
 #pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      float* sk = p.mem + (((size_t)(0 * 2 + m) * p.F + t) * p.H + h) * p.d + c8 * 8;
-      float* sv = p.mem + (((size_t)(1 * 2 + m) * p.F + t) * p.H + h) * p.d + c8 * 8;
-      float k[8], v[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        k[j] = sk[j];
-        v[j] = sv[j];
-      }
-      for (int e = 0; e < p.n_e; ++e) {
-        const int row = p.e_slot[e] * p.F + t;
-        float xk[8], xv[8];
-        unpack8(__ldg(reinterpret_cast<const uint4*>(p.raw_k + ((size_t)h * p.raw_cap + row) * p.d + c8 * 8)), xk);
-        unpack8(__ldg(reinterpret_cast<const uint4*>(p.vc + cache_off(h, planes, p.cap, row, c8))), xv);
-        const bool first = !p.initialised && e == 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          k[j] = first ? xk[j] : __fadd_rn(__fmul_rn(p.a[m], k[j]), __fmul_rn(p.b[m], xk[j]));
-          v[j] = first ? xv[j] : __fadd_rn(__fmul_rn(p.a[m], v[j]), __fmul_rn(p.b[m], xv[j]));
-        }
-      }
-      if (p.n_e > 0) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          sk[j] = k[j];
-          sv[j] = v[j];
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float2 cs = rope_cs(p.rt, c8 * 4 + j, p.tau[m], hr, wc);
-        rot(k[2 * j], k[2 * j + 1], cs.x, cs.y);
-      }
-      const int dst = p.row0 + m * p.F + t;
-      *reinterpret_cast<uint4*>(p.kc + cache_off(h, planes, p.cap, dst, c8)) = pack8(k);
-      *reinterpret_cast<uint4*>(p.vc + cache_off(h, planes, p.cap, dst, c8)) = pack8(v);
+    for (int j = 0; j < 4; ++j) {
+      float2 cs = rope_cs(p.rt, c8 * 4 + j, p.tau[m], hr, wc);
+      rot(k[2 * j], k[2 * j + 1], cs.x, cs.y);
     }
+    const int dst = p.row0 + m * p.F + t;
+    *reinterpret_cast<uint4*>(p.kc + cache_off(h, planes, p.cap, dst, c8)) = pack8(k);
+    *reinterpret_cast<uint4*>(p.vc + cache_off(h, planes, p.cap, dst, c8)) = pack8(v);
   }
 }
 
@@ -333,7 +336,7 @@ cudaError_t launch_rerotate(const RerotateParams& p, cudaStream_t s) {
 }
 
 cudaError_t launch_mem_update(const MemUpdateParams& p, cudaStream_t s) {
-  const int rows = p.F * p.H;
+  const int rows = 2 * p.F * p.H;
   const dim3 block(p.d / 8, 256 / (p.d / 8));
   static int wave = 0;
   int blocks = (rows + block.y - 1) / block.y;
