@@ -14,7 +14,9 @@ follows; the pages are
 
 * rCM page  -- "rCM length extrapolation" guide (dpshk.com, news/6097349):
   strategies 1-5 (Sliding Window, Rolling Sink, Infinity-RoPE, Deep Forcing,
-  Relax Forcing) and the practical tips.
+  Relax Forcing), the MemRoPE tip and the practical tips. Deep Forcing,
+  Relax Forcing and MemRoPE have their own modules (deep_forcing.py,
+  relax_forcing.py, memrope.py), each listing the readings it takes.
 * Causal-Forcing page -- "Causal-Forcing inference walkthrough" (lqnn.cn,
   news/227985): section 3 (KV cache) and section 4 (block-wise denoising).
 * LingBot page -- "LingBot-World 2.0 rolling KV cache" explainer
@@ -33,10 +35,13 @@ from .policy import PolicyOracle, KeptFrame, roll_index
 from .rope import rope_pair_split, rope_angles, rope_apply, token_grid_positions
 from .attention import masked_sdpa, visibility, column_scores, top_c
 from .deep_forcing import DeepForcingOracle, KeptToken
+from .relax_forcing import RelaxForcingOracle
+from .memrope import MemRopeOracle
 from .stream import OracleStream
 
 __all__ = [
     "PolicyOracle", "KeptFrame", "roll_index", "rope_pair_split", "rope_angles",
     "rope_apply", "token_grid_positions", "masked_sdpa", "visibility",
     "column_scores", "top_c", "OracleStream", "DeepForcingOracle", "KeptToken",
+    "RelaxForcingOracle", "MemRopeOracle",
 ]
