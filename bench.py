@@ -495,6 +495,75 @@ def run_hbm(args):
     return 0
 
 
+def run_sdpa_context(args):
+    """Context only (not the product path): torch's own scaled_dot_product_attention
+    on the Wan-1.3B layer-pass shapes against this library's attention on the same
+    shapes, both without an in-chunk mask (torch's fast kernels take no frame mask):
+    one head-major [1, 12, 4680, 128] query block over [1, 12, 29640, 128] keys."""
+    import torch
+    import torch.nn.functional as Fn
+    from rolling_kv_cache_b200 import binding as B
+    from rolling_kv_cache_b200.cache import RollingKVCache
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = rc_synth.WORKLOADS["wan13b"].replace(layers=1, passes=1, mask_block_frames=3)
+    H, d, Nq = w.heads, w.head_dim, w.query_tokens
+    Nk = w.footprint_tokens
+    flops = 4.0 * d * H * Nq * Nk
+
+    def timed(fn, iters=20):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / iters
+
+    g = torch.Generator(device=dev).manual_seed(0)
+    q = torch.randn(1, H, Nq, d, device=dev, dtype=torch.bfloat16, generator=g)
+    k = torch.randn(1, H, Nk, d, device=dev, dtype=torch.bfloat16, generator=g)
+    v = torch.randn(1, H, Nk, d, device=dev, dtype=torch.bfloat16, generator=g)
+    torch_res = {}
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    for name, be in (("cudnn", SDPBackend.CUDNN_ATTENTION), ("flash", SDPBackend.FLASH_ATTENTION),
+                     ("efficient", SDPBackend.EFFICIENT_ATTENTION)):
+        try:
+            with sdpa_kernel([be]):
+                ms = timed(lambda: Fn.scaled_dot_product_attention(q, k, v))
+            torch_res[name] = {"ms": ms, "tflops": flops / (ms / 1e3) / 1e12}
+        except Exception as e:   # backend not available for this shape / build
+            torch_res[name] = {"unavailable": str(e).splitlines()[0][:120]}
+    # this library, steady state of the same stream, the attention kernel's own events
+    cache = RollingKVCache(make_cfg(w, layers=1), dev)
+    pool = [tuple(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+                  for x in rc_synth.chunk_qkv(w, 0, c, 0)) for c in range(3)]
+    out = torch.empty_like(pool[0][0])
+    c = 0
+    for _ in range((w.footprint_frames + 2) // 3 + 3):
+        qq, kk, vv = pool[c % 3]
+        cache.step(0, qq, kk, vv, 3 * c, out=out)
+        c += 1
+    torch.cuda.synchronize()
+    B.rc_profile_begin(cache.handle, 256)
+    for _ in range(20):
+        qq, kk, vv = pool[c % 3]
+        cache.step(0, qq, kk, vv, 3 * c, out=out)
+        c += 1
+    torch.cuda.synchronize()
+    att = B.rc_profile_end(cache.handle)["attention"]
+    ms = att["ms"] / max(1, att["timed"])
+    ours = {"ms": ms, "tflops": att["flops"] / max(1, att["launches"]) / (ms / 1e3) / 1e12}
+    cache.close()
+    print(json.dumps({"metric": "context: attention TFLOP/s on the Wan-1.3B layer-pass shapes, no in-chunk mask",
+                      "unit": "TFLOP/s", "queries": Nq, "keys": Nk, "heads": H, "head_dim": d,
+                      "torch_sdpa": torch_res, "ours": ours}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -509,6 +578,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (small profiling runs)")
+    ap.add_argument("--sdpa-context", action="store_true",
+                    help="context only: torch scaled_dot_product_attention vs this library on the same shapes")
     ap.add_argument("--hbm-cases", default="",
                     help="with --hbm: comma list of cases to run (append, rotcopy, inplace; default all)")
     ap.add_argument("--hbm", action="store_true",
@@ -516,6 +587,8 @@ def main():
     args = ap.parse_args()
     if args.hbm:
         return run_hbm(args)
+    if args.sdpa_context:
+        return run_sdpa_context(args)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     w = rc_synth.WORKLOADS[args.workload]

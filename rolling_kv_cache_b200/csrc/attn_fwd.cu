@@ -189,8 +189,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   volatile int* abort = &abort_sh;
   int dummy_abort = 0;
   volatile int* noabort = reinterpret_cast<volatile int*>(&dummy_abort);
-  Scheduler sc;
-  sc.init(p);
+  Scheduler sc_mem;
+  sc_mem.init(p);
+  // the schedule's state lives in local memory (read once per unit), keeping
+  // registers for the per-tile work
+  Scheduler* volatile sc_ptr = &sc_mem;
+  Scheduler& sc = *sc_ptr;
   Job jb;
 
   if (warp == kProducerWarp && lane == 0) {
