@@ -290,3 +290,29 @@ def test_engine_fuzz_against_oracle():
                 policy=pol_kind, chunk_frames=B_, sink_frames=S_f, window_frames=W_f,
                 chunks=chunks, passes=rng.randint(1, 3), mask_block_frames=rng.randint(1, 3))
         run_stream(w)
+
+
+def test_engine_partial_chunks_sliding_against_oracle():
+    """Sliding / unbounded chunks of 1..chunk_frames frames (the last block of a
+    video, or a caller stepping single frames): state equals the oracle's."""
+    rng = random.Random(77)
+    for trial in range(40):
+        B_ = rng.randint(1, 4)
+        S_f = rng.randint(0, 3)
+        W_f = rng.randint(B_, 10)
+        w = rc_synth.WORKLOADS["tiny"].replace(chunk_frames=B_, sink_frames=S_f, window_frames=W_f)
+        h = B.rc_cache_create(config_for(w, layers=1), 0, 0)
+        pol = PolicyOracle.from_workload(w)
+        g = 0
+        try:
+            for _ in range(rng.randint(1, 20)):
+                n = rng.randint(1, B_)
+                for _pass in range(rng.randint(1, 2)):
+                    B.rc_step(h, 0, 0, 0, 0, g, n, w.policy, 0)
+                    kept = pol.step(g, n)
+                    st = B.rc_get_state(h, 0)
+                    assert lib_kept(st) == oracle_kept(kept)
+                    assert st.chunk_frames == n
+                g += n
+        finally:
+            B.rc_cache_destroy(h)

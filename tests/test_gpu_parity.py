@@ -49,6 +49,22 @@ def test_tiny_every_step(mask_block):
     r.close()
 
 
+@pytest.mark.parametrize("sink,window,grid,heads,d", [
+    (0, 3, (4, 4), 2, 64),      # no sink, window = one chunk: attention over the chunk only
+    (2, 4, (10, 10), 1, 64),    # one history frame, 100-token frames (ragged tiles), one head
+    (1, 6, (3, 50), 3, 128),    # 150-token frames: tiles straddle frame boundaries
+])
+def test_degenerate_and_ragged_configs(sink, window, grid, heads, d):
+    w = W["tiny"].replace(sink_frames=sink, window_frames=window, grid_h=grid[0], grid_w=grid[1],
+                          heads=heads, head_dim=d, chunks=7)
+    r = Runner(w)
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        r.step(c, p)
+        r.check_append_bitexact()
+        r.check_float()
+    r.close()
+
+
 def test_unbounded_policy_equals_full_history():
     w = W["tiny"].replace(policy=rc_synth.POLICY_NONE, window_frames=40, chunks=8)
     r = Runner(w)
