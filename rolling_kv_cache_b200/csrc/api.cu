@@ -605,6 +605,34 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
     at.part_o = split ? c->part_o : nullptr;
     at.part_lse = split ? c->part_lse : nullptr;
     at.n_ctas = split ? G : units;
+    if (split) {
+      // stream-K ranges that level the work: CTA c ran round units c, c + G, ...;
+      // give it the share of the remainder that brings it to the average
+      const long long T_head = at.pair_prefix[NP];
+      auto cum = [&](long long v) { return (v / NP) * T_head + at.pair_prefix[v % NP]; };
+      auto len = [&](long long u) { return (long long)at.pair_prefix[u % NP + 1] - at.pair_prefix[u % NP]; };
+      const long long rounds = units / G;
+      const long long base = cum(rounds * G), W_rem = cum(units) - base;
+      std::vector<double> want(G);
+      double total = (double)W_rem, wsum = 0;
+      for (int cc = 0; cc < G; ++cc) {
+        long long rt = 0;
+        for (long long r = 0; r < rounds; ++r) rt += len(cc + r * G);
+        want[cc] = (double)rt;
+        total += (double)rt;
+      }
+      for (int cc = 0; cc < G; ++cc) {
+        want[cc] = std::max(0.0, total / G - want[cc]);
+        wsum += want[cc];
+      }
+      double acc = 0;
+      for (int cc = 0; cc <= G; ++cc) {
+        at.sk_start[cc] = (int)(base + (wsum > 0 ? (long long)std::floor(W_rem * acc / wsum)
+                                                  : (long long)cc * W_rem / G));
+        if (cc < G) acc += wsum > 0 ? want[cc] : 0;
+      }
+      at.sk_start[G] = (int)(base + W_rem);
+    }
   }
   at.Nq = Nq;
   at.H = H;

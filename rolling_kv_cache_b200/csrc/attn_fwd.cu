@@ -78,9 +78,11 @@ __device__ __forceinline__ int pair_rq_hi(const AttnParams& p, int pair) {
 // tile 0 together, so the query pairs of a head read each K/V tile about
 // when the others do and it comes from DRAM once. The U mod G units left
 // over (the last heads) are then cut stream-K style: their tiles, in (unit,
-// tile) order, are split into G equal ranges, one per CTA; a unit cut
-// between CTAs leaves partial rows for the combine kernel. Their K/V spans
-// only a few heads, so it stays in L2 whatever the offsets.
+// tile) order, are split into G ranges, one per CTA, sized by the host so
+// that every CTA's round tiles plus range tiles come out equal (units differ
+// in length under the in-chunk mask); a unit cut between CTAs leaves partial
+// rows for the combine kernel. Their K/V spans only a few heads, so it stays
+// in L2 whatever the offsets.
 // Without a partial workspace the grid has one CTA per unit.
 struct Scheduler {
   const AttnParams* p;
@@ -105,10 +107,8 @@ struct Scheduler {
     rounds = split ? (int)(U / G) : 1;
     pos = end = 0;
     if (split) {
-      base = cum((long long)rounds * G);
-      const long long W_rem = cum(U) - base;
-      pos = base + (long long)c * W_rem / G;
-      end = base + (long long)(c + 1) * W_rem / G;
+      pos = prm.sk_start[c];
+      end = prm.sk_start[c + 1];
     }
   }
 
@@ -501,8 +501,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
 // lse = log2 sum_i 2^(lse_i). Block (unit, y) takes 32 query rows of the
 // unit; 8 consecutive threads share a row, D/8 columns each, so every warp
 // reads 4 whole rows of a partial at once.
-__device__ __forceinline__ long long owner_of(long long pos, long long W, int G) {
-  return ((pos + 1) * G - 1) / W;  // largest c with floor(c W / G) <= pos
+// The CTA whose stream-K range holds tile position pos: the largest c with
+// sk_start[c] <= pos (empty ranges before it share its start).
+__device__ __forceinline__ int owner_of(const AttnParams& p, int G, long long pos) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.sk_start[mid] <= pos) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
 }
 
 constexpr int kCombineRowsPerBlock = 32;
@@ -518,23 +526,18 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant
   if (u >= U) return;
   const int h = (int)(u / NP), pair = (int)(u % NP);
   auto cum = [&](long long v) { return (v / NP) * T_head + p.pair_prefix[v % NP]; };
-  const long long base = cum(first_rem);
-  const long long W = cum(U) - base;
-  const long long C_u = cum(u) - base;  // unit start in the stream-K range
+  const long long C_u = cum(u);  // unit start (tile position)
   const int T_u = p.pair_prefix[pair + 1] - p.pair_prefix[pair];
-  const int c_lo = (int)owner_of(C_u, W, G), c_hi = (int)owner_of(C_u + T_u - 1, W, G);
+  const int c_lo = owner_of(p, G, C_u), c_hi = owner_of(p, G, C_u + T_u - 1);
   if (c_lo == c_hi) return;  // written directly by one CTA
   const int prow = blockIdx.y * kCombineRowsPerBlock + (threadIdx.x >> 3);
   const int col0 = (threadIdx.x & 7) * kCols;
   const int qtok = pair * 2 * kTileRows + prow;
   if (qtok >= p.Nq) return;
   // slot of CTA c's job on this unit: its first job iff its range starts inside the unit
-  auto slot_of = [&](int cc) {
-    const long long b = (long long)cc * W / G;
-    return 2 * cc + ((b >= C_u) ? 0 : 1);
-  };
-  // a CTA whose stream-K range is empty (fewer remainder tiles than CTAs) holds no part
-  auto has_part = [&](int cc) { return (long long)(cc + 1) * W / G > (long long)cc * W / G; };
+  auto slot_of = [&](int cc) { return 2 * cc + ((p.sk_start[cc] >= C_u) ? 0 : 1); };
+  // a CTA whose stream-K range is empty holds no part
+  auto has_part = [&](int cc) { return p.sk_start[cc + 1] > p.sk_start[cc]; };
   float mx = -INFINITY;
   for (int cc = c_lo; cc <= c_hi; ++cc)
     if (has_part(cc)) mx = fmaxf(mx, p.part_lse[(size_t)slot_of(cc) * 2 * kTileRows + prow]);

@@ -90,6 +90,9 @@ struct alignas(64) AttnParams {
   KvSegment seg[kMaxSegs];
   int n_pairs;                      // query pairs per head (persistent launches)
   int pair_prefix[kMaxPairs + 1];   // KV tiles of pairs [0, q) (same for every head)
+  // stream-K range of CTA c, in (unit, tile) positions: [sk_start[c], sk_start[c + 1]);
+  // sized so that round work + range is the same for every CTA
+  int sk_start[kMaxPersistentCtas + 1];
 };
 
 // K6a: column scores over history tokens (second QK^T pass with final LSE).
