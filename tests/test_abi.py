@@ -111,3 +111,20 @@ def test_rope_tables_are_fp32_roundings_of_fp64():
             assert np.max(np.abs(t[..., 1] - np.sin(a))) < 6e-8
     finally:
         B.rc_cache_destroy(h)
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """No CPU fallback: without librc.so the binding raises instead of
+    computing anything another way."""
+    import importlib
+    import rolling_kv_cache_b200.binding as binding
+    fresh = importlib.reload(binding)
+    try:
+        monkeypatch.setattr(fresh, "LIB_PATH", str(tmp_path / "librc.so"))
+        monkeypatch.setattr(fresh, "_lib", None)
+        with pytest.raises(RuntimeError, match="missing"):
+            fresh.lib()
+        with pytest.raises(RuntimeError):
+            fresh.rc_config_init(1, 2, 64, 16, 1, 6)
+    finally:
+        importlib.reload(binding)
