@@ -195,11 +195,29 @@ def oracle_sample_seconds(w, heads: int, chunk: int = 7):
     return dt, attention_flops(w, n_hist, heads=heads), threads
 
 
+def workload_config(w, world, shard, heads_per_rank):
+    """The JSON line's ``config``: the same for both arms at the same N."""
+    # bytes of one layer's K and V buffers (ring, plus the Deep Forcing region)
+    kv_ring_mb = 2 * heads_per_rank * w.footprint_tokens * w.head_dim * 2 / 1e6
+    return {"workload": w.name, "layers": w.layers, "heads": w.heads,
+            "head_dim": w.head_dim, "frame_seqlen": w.frame_seqlen,
+            "chunk_frames": w.chunk_frames, "sink_frames": w.sink_frames,
+            "window_frames": w.window_frames, "passes_per_chunk": w.passes,
+            "cached_tokens_per_head": w.footprint_tokens,
+            "step": f"one chunk x {w.layers} layers x {w.passes} passes",
+            "parallelism": (f"heads split over {world} GPUs (one stream)" if shard
+                            else f"independent stream per GPU x{world}"),
+            "l2": (f"inputs larger than L2 ({kv_ring_mb:.0f} MB K/V ring per layer"
+                   f"{', %d layers cycled' % w.layers if w.layers > 1 else ''})")}
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     heads = 1
+    shard = args.shard == "heads"
+    heads_per_rank = (w.heads + args.gpus - 1) // args.gpus if shard else w.heads
     for _ in range(args.warmup):
         oracle_sample_seconds(w, heads)
     secs, flops = 0.0, 0.0
@@ -214,7 +232,7 @@ def run_reference(args, w):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name}, "cpu_baseline": {
+            "config": workload_config(w, args.gpus, shard, heads_per_rank), "cpu_baseline": {
                 "value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -326,8 +344,6 @@ def run_ours(args, w):
     prof = B.rc_profile_end(cache.handle)
     cache.device_status()
 
-    # bytes of one layer's K and V buffers (ring, plus the Deep Forcing region)
-    kv_ring_mb = 2 * (h1 - h0) * w.footprint_tokens * w.head_dim * 2 / 1e6
     att = prof["attention"]
     ms_max, flops_total = aggregate_over_ranks(ms, att["flops"], dev)
     value = flops_total / (ms_max / 1e3) / 1e12
@@ -402,16 +418,7 @@ def run_ours(args, w):
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "strong" if shard else "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": w.name, "layers": w.layers, "heads": w.heads,
-                       "head_dim": w.head_dim, "frame_seqlen": w.frame_seqlen,
-                       "chunk_frames": B_, "sink_frames": w.sink_frames,
-                       "window_frames": w.window_frames, "passes_per_chunk": w.passes,
-                       "cached_tokens_per_head": w.footprint_tokens,
-                       "step": f"one chunk x {w.layers} layers x {w.passes} passes",
-                       "parallelism": (f"heads split over {world} GPUs (one stream)" if shard
-                                       else f"independent stream per GPU x{world}"),
-                       "l2": (f"inputs larger than L2 ({kv_ring_mb:.0f} MB K/V ring per layer"
-                              f"{', %d layers cycled' % w.layers if w.layers > 1 else ''})")},
+            "config": workload_config(w, world, shard, h1 - h0),
             "frames_per_s_per_layer": frames_per_s_per_layer,
             "frames_per_s_model": frames / (ms_max / 1e3),
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
