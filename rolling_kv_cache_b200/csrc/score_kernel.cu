@@ -7,21 +7,26 @@
 // second Q K^T pass over the history tiles only (sink and current chunk are
 // not candidates, and every query sees every candidate).
 //
+// The LSE is known before the pass starts, so no row maximum is needed and
+// the pass is computed transposed: S^T = K Q^T puts one key per TMEM lane
+// (M = 128 keys, N = 128 queries), and each thread turns its key's row of
+// S^T into exp2(s c - lse2[q]) and sums it over the queries in registers.
+// There is no P tile, no column-sum GEMM and no exchange between warps.
+//
 // Persistent CTAs walk (head, query pair, KV tile) items in equal contiguous
-// ranges; column sums go to global memory with atomics, so a pair cut
-// between CTAs needs no merge. Per CTA, two 128-query tiles share each K tile:
-//   warps 0-7 / 8-15  softmax of Q0 / Q1: P = 2^(s c - lse2) as bf16 into
-//                     shared memory ([query][key], 128-byte swizzle); each
-//                     warp takes 32 rows x 64 keys, so four softmax warps
-//                     share each SM sub-partition's exp2 unit
-//   warp 16           TMA producer (Q pair per job, K tiles in a 2-stage ring)
+// ranges; the sums go to global memory with atomics, so a pair cut between
+// CTAs needs no merge. Per CTA, two 128-query tiles share each K tile:
+//   warps 0-7 / 8-15  exponentials of Q0 / Q1: warp w reads TMEM lane quarter
+//                     w % 4 (32 keys) and query half (w / 4) % 2 (64 columns),
+//                     so four such warps share each SM sub-partition's exp2
+//                     unit
+//   warp 16           TMA producer (Q pair per job, K tiles in a 3-stage ring)
 //   warps 17 / 18     one MMA issuer per query tile (warp 17 also owns TMEM)
-// The column sum itself runs on the tensor core: D'_g = P_g^T 1 with P_g^T
-// read MN-major from shared memory (M = 128 keys, N = 16, K = 128 queries);
-// lane j of D'_g holds key j's sum over the tile's queries, which group g
-// reads one tile later (its two column halves in turn) and adds to the score
-// buffer.
-// TMEM: S0 [0,128), S1 [128,256), D'_0 [256,288), D'_1 [288,320) (2 buffers each).
+// TMEM: two S^T buffers per query tile, S_g,b at columns [(2g + b) 128, +128):
+// the issuer computes tile t + 1 into one while the exponential warps read
+// tile t from the other. Each job's lse2 (log2 units, +inf past the last
+// query) is staged in shared memory by the exponential warps, one buffer per
+// job parity.
 // Bounded waits (RC_ETIMEOUT in the status word), no trap.
 #include "attn_common.cuh"
 #include "kernels.cuh"
@@ -35,24 +40,20 @@ constexpr int kSoftmaxWarps = 16;
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;  // and 18
 constexpr int kScoreThreads = 19 * 32;
-constexpr uint32_t kPTileBytes = 128 * 128 * 2;  // P: 128 queries x 128 keys bf16
-constexpr uint32_t kOnesBytes = 16 * 128 * 2;    // B = ones: 16 x 128 bf16
+constexpr int kKStages = 3;
 
 template <int D>
 struct ScoreLayout {
   static constexpr int kSub = D / 64;
   static constexpr uint32_t kTile = kSubTileBytes * kSub;  // Q or K tile: 128 rows x D
   static constexpr uint32_t kQ = 0;                         // Q0, Q1
-  static constexpr uint32_t kK = 2 * kTile;                 // 2 stages
-  static constexpr uint32_t kP = 4 * kTile;                 // P0, P1
-  static constexpr uint32_t kOnes = kP + 2 * kPTileBytes;
-  static constexpr uint32_t kBytes = kOnes + kOnesBytes;
+  static constexpr uint32_t kK = 2 * kTile;                 // kKStages stages
+  static constexpr uint32_t kBytes = kK + kKStages * kTile;
   static constexpr uint32_t kDynSmem = kBytes + 1024;
 };
 
 struct ScoreJob {
   int h, q0, kv_lo, kv_hi;
-  bool has1;
 };
 
 // Equal contiguous ranges of the W = H * NP * T work items (head, pair, tile).
@@ -65,6 +66,8 @@ struct ScoreScheduler {
     pos = (long long)blockIdx.x * W / gridDim.x;
     end = (long long)(blockIdx.x + 1) * W / gridDim.x;
   }
+  // Both query tiles of a pair always run: rows past Nq load as zeros and
+  // get lse2 = +inf, so their terms are exactly 0.
   __device__ bool next(ScoreJob& j) {
     if (pos >= end) return false;
     const long long unit = pos / p->tiles;
@@ -75,42 +78,32 @@ struct ScoreScheduler {
     j.q0 = (int)(unit % p->n_pairs) * 2 * kTileRows;
     j.kv_lo = off;
     j.kv_hi = off + len;
-    // both tiles always: rows past Nq load as zeros and get lse2 = +inf, so
-    // their P is exactly 0 (keeps the two issuers' barrier phases in step)
-    j.has1 = true;
     return true;
   }
 };
 
-// P = 2^(s c - lse2) of 32 keys of one row (S columns c0 .. c0 + 31 of this
-// warp's half) as bf16, into the row's four 16-byte chunks c0/8 .. c0/8 + 3 of
-// the 128-byte-swizzled sub-tile. Keys at or past lim (ragged tile end) get 0.
-template <bool kCheck>
-__device__ __forceinline__ void exp_store(const uint32_t (&r)[32], int c0, int lim, float c, float lse2,
-                                          uint8_t* sProw, int row) {
-  uint32_t pk[16];
+// Sum over 32 queries of exp2(s c - lse2): r holds S^T columns (queries)
+// q .. q + 31 of this thread's key, lse the matching lse2 values.
+__device__ __forceinline__ float exp_sum32(const uint32_t (&r)[32], const float* lse, float c) {
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    float a = ptx::ex2(fmaf(__uint_as_float(r[2 * k]), c, -lse2));
-    float b = ptx::ex2(fmaf(__uint_as_float(r[2 * k + 1]), c, -lse2));
-    if (kCheck) {
-      if (c0 + 2 * k >= lim) a = 0.f;
-      if (c0 + 2 * k + 1 >= lim) b = 0.f;
-    }
-    pk[k] = ptx::pack_bf16x2(a, b);
+  for (int k = 0; k < 32; k += 4) {
+    const float4 l = *reinterpret_cast<const float4*>(lse + k);
+    a0 += ptx::ex2(fmaf(__uint_as_float(r[k + 0]), c, -l.x));
+    a1 += ptx::ex2(fmaf(__uint_as_float(r[k + 1]), c, -l.y));
+    a2 += ptx::ex2(fmaf(__uint_as_float(r[k + 2]), c, -l.z));
+    a3 += ptx::ex2(fmaf(__uint_as_float(r[k + 3]), c, -l.w));
   }
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-    *reinterpret_cast<uint4*>(sProw + (((c0 / 8 + q) ^ (row & 7)) << 4)) =
-        make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+  return (a0 + a1) + (a2 + a3);
 }
 
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const __grid_constant__ ScoreParams p) {
   using L = ScoreLayout<D>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_q, bar_qe, bar_kf[2], bar_ke[2], bar_s[2], bar_sfree[2], bar_p[2], bar_pfree[2],
-      bar_dfull[2][2], bar_dfree[2][2], bar_fin[2];
+  __shared__ uint64_t bar_q, bar_qe, bar_kf[kKStages], bar_ke[kKStages], bar_s[2][2], bar_sfree[2][2],
+      bar_lse[2], bar_fin[2];
+  __shared__ __align__(16) float s_lse[2][2][kTileRows];  // [job parity][query tile][query]
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -118,25 +111,20 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const __grid_co
   const uint32_t base_u32 = (ptx::smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_u32 - ptx::smem_u32(smem_raw));
 
-  // B operand of the column sum: all ones (layout-free)
-  for (uint32_t i = threadIdx.x; i < kOnesBytes / 4; i += blockDim.x)
-    reinterpret_cast<uint32_t*>(base + L::kOnes)[i] = 0x3F803F80u;
-  ptx::fence_proxy_async_smem();
   if (threadIdx.x == 0) {
     ptx::mbar_init(&bar_q, 1);
     ptx::mbar_init(&bar_qe, 2);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kKStages; ++i) {
       ptx::mbar_init(&bar_kf[i], 1);
       ptx::mbar_init(&bar_ke[i], 2);
-      ptx::mbar_init(&bar_s[i], 1);
-      ptx::mbar_init(&bar_sfree[i], 256);
-      ptx::mbar_init(&bar_p[i], 256);
-      ptx::mbar_init(&bar_pfree[i], 1);
+    }
+    for (int g = 0; g < 2; ++g) {
       for (int b = 0; b < 2; ++b) {
-        ptx::mbar_init(&bar_dfull[i][b], 1);
-        ptx::mbar_init(&bar_dfree[i][b], 128);
+        ptx::mbar_init(&bar_s[g][b], 1);
+        ptx::mbar_init(&bar_sfree[g][b], 256);
       }
-      ptx::mbar_init(&bar_fin[i], 1);
+      ptx::mbar_init(&bar_lse[g], 256);
+      ptx::mbar_init(&bar_fin[g], 1);
     }
     abort_sh = 0;
     ptx::fence_mbar_init();
@@ -158,12 +146,12 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const __grid_co
 
   if (warp == kProducerWarp && lane == 0) {
     // ---------------------------------------------------------- producer
-    int nq = 0, g = 0, nk[2] = {0, 0};
+    int nq = 0, g = 0, nk[kKStages] = {0, 0, 0};
     bool ok = true;
     while (ok && sc.next(jb)) {
       if (nq > 0 && !ptx::mbar_wait(&bar_qe, (nq - 1) & 1, abort, p.status, RC_ETIMEOUT)) break;
-      ptx::mbar_arrive_expect_tx(&bar_q, (jb.has1 ? 2 : 1) * L::kTile);
-      for (int i = 0; i < (jb.has1 ? 2 : 1); ++i)
+      ptx::mbar_arrive_expect_tx(&bar_q, 2 * L::kTile);
+      for (int i = 0; i < 2; ++i)
         for (int k = 0; k < L::kSub; ++k)
           ptx::tma_load_3d(&p.tm_q, &bar_q, base + L::kQ + i * L::kTile + k * kSubTileBytes, 64 * k,
                            jb.q0 + i * kTileRows, jb.h);
@@ -172,8 +160,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const __grid_co
       wk.seek(jb.kv_lo);
       Tile t;
       for (int j = jb.kv_lo; j < jb.kv_hi && wk.next(t); ++j, ++g) {
-        const int st = g & 1;
-        if (g >= 2 && !ptx::mbar_wait(&bar_ke[st], ((g >> 1) - 1) & 1, abort, p.status, RC_ETIMEOUT)) {
+        const int st = g % kKStages, use = g / kKStages;
+        if (use > 0 && !ptx::mbar_wait(&bar_ke[st], (use - 1) & 1, abort, p.status, RC_ETIMEOUT)) {
           ok = false;
           break;
         }
@@ -184,144 +172,97 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const __grid_co
         nk[st]++;
       }
     }
+    // copies still in flight complete before the CTA leaves
     if (nq) ptx::mbar_wait(&bar_q, (nq - 1) & 1, noabort, p.status, RC_ETIMEOUT);
-    for (int st = 0; st < 2; ++st)
+    for (int st = 0; st < kKStages; ++st)
       if (nk[st]) ptx::mbar_wait(&bar_kf[st], (nk[st] - 1) & 1, noabort, p.status, RC_ETIMEOUT);
   } else if ((warp == kMmaWarp || warp == kMmaWarp + 1) && lane == 0) {
     // ---------------------------------------------------------- MMA issuers
     // one thread per query tile, so the two groups' pipelines never wait on
-    // each other; K stages and the Q pair are released by both (count 2)
+    // each other; K stages and the Q pair are released by both (count 2).
+    // S^T(t) = K(t) Q_g^T goes to buffer t & 1 once the exponential warps
+    // have read tile t - 2 from it.
     const int g = warp - kMmaWarp;
-    constexpr uint32_t idesc_s = ptx::idesc_bf16(128, 128, 0, 0);
-    constexpr uint32_t idesc_c = ptx::idesc_bf16(128, 16, 1, 0);  // A = P^T (MN-major), B = ones (K-major)
+    constexpr uint32_t idesc = ptx::idesc_bf16(128, 128, 0, 0);
     const uint32_t sQg = base_u32 + L::kQ + g * L::kTile;
-    const uint32_t sP = base_u32 + L::kP + g * kPTileBytes;
-    const uint32_t sOnes = base_u32 + L::kOnes;
-    auto issue_s = [&](int st) {
-      const uint32_t sK = base_u32 + L::kK + st * L::kTile;
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const uint32_t off = (ks >> 2) * kSubTileBytes + (ks & 3) * 32;
-        ptx::mma_ss(tmem + g * 128, ptx::sdesc_sw128(sQg + off, 16, 1024), ptx::sdesc_sw128(sK + off, 16, 1024),
-                    idesc_s, ks > 0);
-      }
-      ptx::mma_commit(&bar_s[g]);
-    };
-    int nq = 0, gk = 0, gt = 0, gd = 0;
+    const uint32_t tSg = tmem + g * 256;
+    int nq = 0, gk = 0, t = 0;  // Q pairs waited for, K tiles consumed, S tiles issued
     bool ok = true;
     while (ok && sc.next(jb)) {
-      const int n = jb.kv_hi - jb.kv_lo;
       if (!ptx::mbar_wait(&bar_q, nq & 1, abort, p.status, RC_ETIMEOUT)) break;
       ++nq;
-      if (!ptx::mbar_wait(&bar_kf[gk & 1], (gk >> 1) & 1, abort, p.status, RC_ETIMEOUT)) break;
-      if (gt > 0 && !ptx::mbar_wait(&bar_sfree[g], (gt - 1) & 1, abort, p.status, RC_ETIMEOUT)) break;
-      ptx::tc_fence_after();
-      issue_s(gk & 1);
-      ptx::mma_commit(&bar_ke[gk & 1]);
-      if (n == 1) ptx::mma_commit(&bar_qe);
-      for (int j = 0; j < n; ++j, ++gk, ++gt, ++gd) {
-        if (j + 1 < n) {  // S of the next tile once this one's S has been read
-          const int st1 = (gk + 1) & 1;
-          if (!ptx::mbar_wait(&bar_kf[st1], ((gk + 1) >> 1) & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
-          if (!ptx::mbar_wait(&bar_sfree[g], gt & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
-          ptx::tc_fence_after();
-          issue_s(st1);
-          ptx::mma_commit(&bar_ke[st1]);
-          if (j + 2 == n) ptx::mma_commit(&bar_qe);
-        }
-        const int db = gd & 1;
-        if (gd >= 2 && !ptx::mbar_wait(&bar_dfree[g][db], ((gd >> 1) - 1) & 1, abort, p.status, RC_ETIMEOUT)) {
+      const int n = jb.kv_hi - jb.kv_lo;
+      for (int j = 0; j < n; ++j, ++gk, ++t) {
+        const int st = gk % kKStages, b = t & 1;
+        if (!ptx::mbar_wait(&bar_kf[st], (gk / kKStages) & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
+        if (t >= 2 && !ptx::mbar_wait(&bar_sfree[g][b], ((t >> 1) - 1) & 1, abort, p.status, RC_ETIMEOUT)) {
           ok = false;
           break;
         }
-        if (!ptx::mbar_wait(&bar_p[g], gt & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
         ptx::tc_fence_after();
+        const uint32_t sK = base_u32 + L::kK + st * L::kTile;
 #pragma unroll
-        for (int ks = 0; ks < kTileRows / 16; ++ks)
-          ptx::mma_ss(tmem + 256 + g * 32 + db * 16, ptx::sdesc_sw128(sP + ks * 2048, kSubTileBytes, 1024),
-                      ptx::sdesc_sw128(sOnes + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024), idesc_c, ks > 0);
-        ptx::mma_commit(&bar_pfree[g]);
-        ptx::mma_commit(&bar_dfull[g][db]);
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * kSubTileBytes + (ks & 3) * 32;
+          ptx::mma_ss(tSg + b * 128, ptx::sdesc_sw128(sK + off, 16, 1024), ptx::sdesc_sw128(sQg + off, 16, 1024),
+                      idesc, ks > 0);
+        }
+        ptx::mma_commit(&bar_s[g][b]);
+        ptx::mma_commit(&bar_ke[st]);
+        if (j + 1 == n) ptx::mma_commit(&bar_qe);
       }
     }
     ptx::mma_commit(&bar_fin[g]);
     ptx::mbar_wait(&bar_fin[g], 0, noabort, p.status, RC_ETIMEOUT);
   } else if (warp < kSoftmaxWarps) {
-    // ---------------------------------------------------------- softmax
-    // group g = warp / 8 owns query tile g; within it warp w reads TMEM lane
-    // quarter w % 4 (rows) and column half (w / 4) % 2 (keys [64 ch, 64 ch + 64))
+    // ---------------------------------------------------------- exponentials
     const int grp = warp >> 3;
     const int ch = (warp >> 2) & 1;
     const int wq = warp & 3;
-    const int row = wq * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + grp * 128 + ch * 64;
-    uint8_t* sProw = base + L::kP + grp * kPTileBytes + ch * kSubTileBytes + row * 128;
+    const int key = wq * 32 + lane;  // TMEM lane = key within the tile
+    const uint32_t tSg = tmem + (static_cast<uint32_t>(wq * 32) << 16) + grp * 256 + ch * 64;
     const float c = p.scale_log2;
-    int gs = 0;            // this group's tiles (phases of s / sfree / p / pfree)
-    int gd = 0;            // D' sums of this group (drained by the two column halves in turn)
-    int prev_tok = 0, prev_nvalid = 0;
-    bool have_prev = false;
-    // add the previous tile's key sums (lane j of this group's D' = key j) to the scores
-    auto drain = [&]() -> bool {
-      if (!have_prev) return true;
-      have_prev = false;
-      const int db = gd & 1;  // buffer db is drained by column half db
-      const uint32_t phase = (gd >> 1) & 1;
-      ++gd;
-      if (db != ch) return true;
-      if (!ptx::mbar_wait(&bar_dfull[grp][db], phase, abort, p.status, RC_ETIMEOUT)) return false;
-      ptx::tc_fence_after();
-      const uint32_t v = ptx::tmem_ld1(tmem + lane_off + 256 + grp * 32 + db * 16);
-      ptx::tmem_ld_wait();
-      if (row < prev_nvalid) atomicAdd(p.score_phys + prev_tok + row, __uint_as_float(v));
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bar_dfree[grp][db]);
-      return true;
-    };
+    int gs = 0;  // this group's tiles read so far
+    int nj = 0;  // jobs so far (lse2 buffer parity)
     bool ok = true;
     while (ok && sc.next(jb)) {
       if (*abort) break;
-      const int qtok = jb.q0 + grp * kTileRows + row;
-      const float lse2 = qtok < p.Nq ? p.lse[(size_t)jb.h * p.Nq + qtok] * 1.4426950408889634f : INFINITY;
+      // this job's lse2, written by the first column half (one query each)
+      float* lse = s_lse[nj & 1][grp];
+      if (ch == 0) {
+        const int qtok = jb.q0 + grp * kTileRows + key;
+        lse[key] = qtok < p.Nq ? p.lse[(size_t)jb.h * p.Nq + qtok] * 1.4426950408889634f : INFINITY;
+      }
+      ptx::mbar_arrive(&bar_lse[grp]);
+      if (!ptx::mbar_wait(&bar_lse[grp], nj & 1, abort, p.status, RC_ETIMEOUT)) break;
+      ++nj;
+      const float* lse_h = lse + ch * 64;
       TileWalker wk{p.seg, p.n_segs, 0x7fffffff};
       wk.seek(jb.kv_lo);
       Tile t;
-      for (int j = jb.kv_lo; j < jb.kv_hi && wk.next(t); ++j) {
-        if (!ptx::mbar_wait(&bar_s[grp], gs & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
+      for (int j = jb.kv_lo; j < jb.kv_hi && wk.next(t); ++j, ++gs) {
+        const int b = gs & 1;
+        if (!ptx::mbar_wait(&bar_s[grp][b], (gs >> 1) & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
         ptx::tc_fence_after();
-        // P smem of the previous tile must have been read by its column-sum MMA
-        if (gs > 0 && !ptx::mbar_wait(&bar_pfree[grp], (gs - 1) & 1, abort, p.status, RC_ETIMEOUT)) {
-          ok = false;
-          break;
-        }
-        const int lim = t.nvalid - ch * 64;  // valid keys in this half
+        const uint32_t tS = tSg + b * 128;
+        float sum;
         {
           uint32_t r[32];
           ptx::tmem_ld32(tS, r);
           ptx::tmem_ld_wait();
-          if (lim >= 64) exp_store<false>(r, 0, lim, c, lse2, sProw, row);
-          else exp_store<true>(r, 0, lim, c, lse2, sProw, row);
+          sum = exp_sum32(r, lse_h, c);
         }
         {
           uint32_t r[32];
           ptx::tmem_ld32(tS + 32, r);
           ptx::tmem_ld_wait();
           ptx::tc_fence_before();
-          ptx::mbar_arrive(&bar_sfree[grp]);  // S read: the MMA may overwrite it
-          if (lim >= 64) exp_store<false>(r, 32, lim, c, lse2, sProw, row);
-          else exp_store<true>(r, 32, lim, c, lse2, sProw, row);
+          ptx::mbar_arrive(&bar_sfree[grp][b]);  // S^T read: the next-but-one tile may overwrite it
+          sum += exp_sum32(r, lse_h + 32, c);
         }
-        ptx::fence_proxy_async_smem();
-        ptx::mbar_arrive(&bar_p[grp]);
-        ++gs;
-        if (!drain()) { ok = false; break; }
-        prev_tok = t.tok;
-        prev_nvalid = t.nvalid;
-        have_prev = true;
+        if (key < t.nvalid) atomicAdd(p.score_phys + t.tok + key, sum);
       }
     }
-    if (ok) drain();
   }
   ptx::tc_fence_before();
   __syncthreads();
