@@ -190,8 +190,10 @@ def _topc_checks(w, r, ref):
             assert abs(sr[pos[c]] - kth) <= 1e-3 * max(1.0, kth)
 
 
-def test_infinity_rope_small_with_scores():
-    w = W["infinity_rope"].replace(heads=2, grid_h=8, grid_w=8, chunks=18, cut_chunks=(9, 13), topc=100)
+@pytest.mark.parametrize("d", [128, 64])
+def test_infinity_rope_small_with_scores(d):
+    w = W["infinity_rope"].replace(heads=2, head_dim=d, grid_h=8, grid_w=8, chunks=18, cut_chunks=(9, 13),
+                                   topc=100)
     r = Runner(w)
     for c, p, g0, cut in rc_synth.stream_schedule(w):
         r.step(c, p, cut, scores=True)
