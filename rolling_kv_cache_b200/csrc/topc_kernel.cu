@@ -8,6 +8,13 @@
 // selected logical indices in index order, taking every score above the
 // threshold and the lowest-index ties at it. Output is ascending; missing
 // entries (fewer candidates than C) are -1.
+// The scores of one step share their top bytes, so a warp adds the count of
+// its lanes that fall in the first valid lane's bin with one atomic (the
+// rest add their own); one warp finds the threshold digit by a shuffle scan
+// over the 256 bins; the compaction gives each thread a contiguous run of
+// candidates and places them with one block scan of (above, tied) counts:
+// the selected elements before a thread are the above ones plus
+// min(ties before it, ties taken).
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -22,28 +29,29 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// Exclusive block-wide scan of one int per thread; returns the block total.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
+// Exclusive block-wide scan of one 64-bit value per thread; returns the
+// block total in `total`.
+__device__ __forceinline__ long long block_exclusive_scan(long long v, long long* warp_tot, long long& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
+  long long x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, x, o);
+    const long long y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
   if (lane == 31) warp_tot[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int w = warp_tot[lane];
+    long long w = warp_tot[lane];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, w, o);
+      const long long y = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += y;
     }
     warp_tot[lane] = w;  // inclusive over warps
   }
   __syncthreads();
-  const int before = (warp > 0 ? warp_tot[warp - 1] : 0) + x - v;
+  const long long before = (warp > 0 ? warp_tot[warp - 1] : 0) + x - v;
   total = warp_tot[31];
   __syncthreads();
   return before;
@@ -51,10 +59,11 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& t
 
 __global__ void __launch_bounds__(kTopcThreads) topc_kernel(const __grid_constant__ TopCParams p) {
   __shared__ int hist[256];
-  __shared__ int warp_tot[32];
+  __shared__ long long warp_tot[32];
   __shared__ uint32_t sh_prefix, sh_mask;
   __shared__ int sh_k;
   const int n = p.n_cand_frames * p.F;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float* lg = p.scores_out;
   for (int i = threadIdx.x; i < n; i += kTopcThreads) {
     const int fi = i / p.F, t = i - fi * p.F;
@@ -74,43 +83,84 @@ __global__ void __launch_bounds__(kTopcThreads) topc_kernel(const __grid_constan
       for (int i = threadIdx.x; i < 256; i += kTopcThreads) hist[i] = 0;
       __syncthreads();
       const uint32_t prefix = sh_prefix, mask = sh_mask;
-      for (int i = threadIdx.x; i < n; i += kTopcThreads) {
-        const uint32_t key = order_key(lg[i]);
-        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
-      }
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        int k = sh_k, cum = 0, d = 255;
-        for (; d > 0; --d) {
-          if (cum + hist[d] >= k) break;
-          cum += hist[d];
+      // whole warps step together (b is warp-uniform) so the votes see every lane
+      for (int b = warp * 32; b < n; b += kTopcThreads) {
+        const int i = b + lane;
+        int digit = -1;
+        if (i < n) {
+          const uint32_t key = order_key(lg[i]);
+          if ((key & mask) == prefix) digit = (int)((key >> shift) & 255u);
         }
-        sh_k = k - cum;
-        sh_prefix = prefix | (static_cast<uint32_t>(d) << shift);
-        sh_mask = mask | (255u << shift);
+        const uint32_t valid = __ballot_sync(0xffffffffu, digit >= 0);
+        if (valid == 0) continue;
+        const int src = __ffs(valid) - 1;
+        const int lead = __shfl_sync(0xffffffffu, digit, src);
+        const uint32_t same = __ballot_sync(0xffffffffu, digit == lead);
+        if (lane == src) atomicAdd(&hist[lead], __popc(same));
+        else if (digit >= 0 && digit != lead) atomicAdd(&hist[digit], 1);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane l holds bins 255 - 8 l - j (j = 0..7): counts from the top
+        int cnt[8], tot = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          cnt[j] = hist[255 - 8 * lane - j];
+          tot += cnt[j];
+        }
+        int incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const int excl = incl - tot;
+        const int k = sh_k;
+        // the first bin, from the top, at which the running count reaches k
+        // (bin 0 if none does)
+        const uint32_t hit = __ballot_sync(0xffffffffu, excl < k && k <= incl);
+        const int hl = hit ? __ffs(hit) - 1 : 31;
+        if (lane == hl) {
+          int cum = excl, d = 0;
+          for (int j = 0; j < 8; ++j) {
+            d = 255 - 8 * lane - j;
+            if (cum + cnt[j] >= k || d == 0) break;
+            cum += cnt[j];
+          }
+          sh_k = k - cum;
+          sh_prefix = prefix | (static_cast<uint32_t>(d) << shift);
+          sh_mask = mask | (255u << shift);
+        }
       }
       __syncthreads();
     }
-  }
-  const uint32_t thr = sh_prefix;
-  const int k_eq = sh_k;  // ties at the threshold to take, lowest index first
-  int eq_base = 0, out_base = 0;
-  for (int c0 = 0; c0 < n && take > 0; c0 += kTopcThreads) {
-    const int i = c0 + threadIdx.x;
-    uint32_t key = 0;
-    if (i < n) key = order_key(lg[i]);
-    const int gt = (i < n && key > thr) ? 1 : 0;
-    const int eq = (i < n && key == thr) ? 1 : 0;
-    int eq_tot, sel_tot;
-    const int eq_rank = eq_base + block_exclusive_scan(eq, warp_tot, eq_tot);
-    const int sel = gt || (eq && eq_rank < k_eq);
-    const int pos = out_base + block_exclusive_scan(sel, warp_tot, sel_tot);
-    if (sel && pos < p.C) {
-      const int fi = i / p.F, t = i - fi * p.F;
-      p.topc[pos] = p.cand_lpos[fi] * p.F + t;
+    const uint32_t thr = sh_prefix;
+    const int k_eq = sh_k;  // ties at the threshold to take, lowest index first
+    const int per = (n + kTopcThreads - 1) / kTopcThreads;
+    const int i0 = min(n, threadIdx.x * per), i1 = min(n, i0 + per);
+    int gt = 0, eq = 0;
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t key = order_key(lg[i]);
+      gt += key > thr;
+      eq += key == thr;
     }
-    eq_base += eq_tot;
-    out_base += sel_tot;
+    long long tot;
+    const long long before = block_exclusive_scan(((long long)gt << 32) | (long long)eq, warp_tot, tot);
+    const int gt_before = (int)(before >> 32), eq_before = (int)(before & 0xffffffffll);
+    int pos = gt_before + min(eq_before, k_eq);
+    int eq_seen = eq_before;
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t key = order_key(lg[i]);
+      bool sel = key > thr;
+      if (key == thr) sel = eq_seen++ < k_eq;
+      if (sel) {
+        if (pos < p.C) {
+          const int fi = i / p.F, t = i - fi * p.F;
+          p.topc[pos] = p.cand_lpos[fi] * p.F + t;
+        }
+        ++pos;
+      }
+    }
   }
   for (int i = take + threadIdx.x; i < p.C; i += kTopcThreads) p.topc[i] = -1;
 }

@@ -137,3 +137,37 @@ def test_scores_and_topc_on_stream():
             assert out["scores"].sum() < w.heads * w.query_tokens
             assert list(out["topc"]) == sorted(out["topc"])
             assert len(out["topc"]) == min(w.topc, n_hist)
+
+
+def _bf16_round(x):
+    a = np.asarray(x, dtype=np.float32)
+    b = a.view(np.uint32).astype(np.uint64)
+    r = ((b + 0x7FFF + ((b >> 16) & 1)) >> 16) << 16   # round to nearest even
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_score_tolerance_covers_bf16_storage(d, monkeypatch):
+    """The GPU parity bar for token scores (SCORE_TOL of the largest) against
+    what storing the rotated queries and keys in bf16 alone does to the fp64
+    scores on the score parity stream (Infinity-RoPE, two RoPE cuts): the
+    bar must sit above that, with room for the fp32 arithmetic and the
+    in-place re-rotations, and within a small factor of it."""
+    import oracle.stream as stream_mod
+    from rcutil import SCORE_TOL
+    w = rc_synth.WORKLOADS["infinity_rope"].replace(heads=2, head_dim=d, grid_h=8, grid_w=8, chunks=18,
+                                                   cut_chunks=(9, 13), topc=100)
+    o = OracleStream(w)
+    worst = 0.0
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        if cut:
+            o.reindex(1 | 2, w.cut_delta)
+        o.step(c, p)
+        monkeypatch.setattr(stream_mod, "rope_apply", rope_apply)
+        exact = o.outputs(want_scores=True)["scores"]
+        monkeypatch.setattr(stream_mod, "rope_apply", lambda x, ang: _bf16_round(rope_apply(x, ang)))
+        stored = o.outputs(want_scores=True)["scores"]
+        if len(exact):
+            worst = max(worst, np.max(np.abs(exact - stored)) / max(1.0, np.max(np.abs(exact))))
+    assert worst > 0.0
+    assert 1.5 * worst <= SCORE_TOL <= 8 * worst, (worst, SCORE_TOL)
