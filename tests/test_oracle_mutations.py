@@ -109,3 +109,119 @@ def test_lingbot_pin_rejects_window_off_by_one():
             return super()._sliding(g0, n, window + 1)
     with pytest.raises(AssertionError):
         pins.check_lingbot_numbers(Wider, 1560, 6, 12, 3, 30)
+
+
+# ---- the policy oracles of the next rows: each pinned test file must reject
+# a copy of its oracle with a plausible mistake planted.
+
+import oracle.deep_forcing as odf
+import oracle.memrope as omr
+import oracle.relax_forcing as orf
+
+import test_oracle_deep_forcing as tdf
+import test_oracle_memrope as tmr
+import test_oracle_relax_forcing as trf
+
+
+def _rejected(*checks):
+    """True when at least one of the pinned checks fails."""
+    for fn, args in checks:
+        try:
+            fn(*args)
+        except AssertionError:
+            return True
+    return False
+
+
+def test_deep_forcing_pins_reject_region_time_off_by_one(monkeypatch):
+    orig = odf.DeepForcingOracle.kept
+
+    def kept(self):
+        return [odf.KeptToken(k.content, k.tok, k.tau - 1, k.region, k.rank) if k.region == "comp" else k
+                for k in orig(self)]
+    monkeypatch.setattr(odf.DeepForcingOracle, "kept", kept)
+    assert _rejected((tdf.test_hand_enumerated_stream, ()))
+
+
+def test_deep_forcing_pins_reject_pool_without_leaving_frames(monkeypatch):
+    # the pool forgets the frames leaving the tail: only the old region is ever re-selected
+    orig_step = odf.DeepForcingOracle.step
+
+    def step(self, frame_start, n_frames, pool_scores=None, selection=None):
+        if self.cur_start is not None and frame_start == self.cur_start:
+            return orig_step(self, frame_start, n_frames, pool_scores, selection)
+        self.end = frame_start + n_frames
+        self.cur_start, self.cur_n = frame_start, n_frames
+        self.last_selection = None
+        return self.kept()
+    monkeypatch.setattr(odf.DeepForcingOracle, "step", step)
+    assert _rejected((tdf.test_hand_enumerated_stream, ()))
+
+
+def test_deep_forcing_pins_reject_ties_to_the_newer_token(monkeypatch):
+    def ties_high(scores, idx, C):
+        order = np.lexsort((-np.asarray(idx), -np.asarray(scores)))
+        return np.sort(np.asarray(idx)[order[:C]])
+    monkeypatch.setattr(odf, "top_c", ties_high)
+    assert _rejected((tdf.test_hand_enumerated_stream, ()))
+
+
+def test_relax_forcing_pins_reject_complement_sign(monkeypatch):
+    def scores(pool_desc, tail_desc, weight):
+        n = len(pool_desc)
+        align = np.array([orf.cosine(d, tail_desc) for d in pool_desc])
+        comp = np.ones(n)
+        if n > 1:
+            for i in range(n):
+                comp[i] = 1.0 + sum(orf.cosine(pool_desc[i], pool_desc[j]) for j in range(n) if j != i) / (n - 1)
+        return weight * align + (1.0 - weight) * comp
+    monkeypatch.setattr(orf, "relax_scores", scores)
+    assert _rejected((trf.test_hand_computed_stream, (0.5,)), (trf.test_hand_computed_stream, (0.9,)))
+
+
+def test_relax_forcing_pins_reject_swapped_weights(monkeypatch):
+    orig = orf.relax_scores
+    monkeypatch.setattr(orf, "relax_scores", lambda p, t, w: orig(p, t, 1.0 - w))
+    assert _rejected((trf.test_hand_computed_stream, (0.9,)))
+
+
+def test_relax_forcing_pins_reject_ties_to_the_newer_frame(monkeypatch):
+    def select(scores, K):
+        order = sorted(range(len(scores)), key=lambda i: (-scores[i], -i))
+        return sorted(order[:K])
+    monkeypatch.setattr(orf, "select_frames", select)
+    assert _rejected((trf.test_hand_computed_stream, (0.5,)), (trf.test_hand_computed_stream, (0.9,)))
+
+
+def test_memrope_pins_reject_swapped_ema_weights(monkeypatch):
+    class Swapped(omr.MemRopeOracle):
+        def __init__(self, *a, **kw):
+            super().__init__(*a, **kw)
+            self.alpha = {m: 1.0 - v for m, v in self.alpha.items()}
+    monkeypatch.setattr(tmr, "MemRopeOracle", Swapped)
+    assert _rejected((tmr.test_hand_computed_memories, ()))
+
+
+def test_memrope_pins_reject_long_memory_inside_the_sink(monkeypatch):
+    orig = omr.MemRopeOracle.kept
+
+    def kept(self):
+        return [odf.KeptToken(k.content, k.tok, k.tau - 1, k.region, k.rank) if k.content == omr.MEM_LONG else k
+                for k in orig(self)]
+    monkeypatch.setattr(omr.MemRopeOracle, "kept", kept)
+    assert _rejected((tmr.test_hand_computed_memories, ()))
+
+
+def test_memrope_pins_reject_zero_initialised_memories(monkeypatch):
+    # the first evicted frame folded into zero memories instead of initialising them
+    orig_step = omr.MemRopeOracle.step
+
+    def step(self, frame_start, n_frames):
+        for m in (omr.MEM_LONG, omr.MEM_SHORT):
+            if self.mem_k[m] is None:
+                xk = self.raw_frame(0, 1)
+                self.mem_k[m] = np.zeros_like(xk)
+                self.mem_v[m] = np.zeros_like(self.raw_frame(0, 2))
+        return orig_step(self, frame_start, n_frames)
+    monkeypatch.setattr(omr.MemRopeOracle, "step", step)
+    assert _rejected((tmr.test_hand_computed_memories, ()), (tmr.test_ema_closed_form_and_extremes, (0.3,)))
