@@ -128,3 +128,43 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
             fresh.rc_config_init(1, 2, 64, 16, 1, 6)
     finally:
         importlib.reload(binding)
+
+
+def _limit_cfg(policy, sink, window, chunk=3, **over):
+    cfg = B.rc_config_init(1, 2, 64, 16, sink, window)
+    cfg.chunk_frames = chunk
+    cfg.policy = policy
+    for k, v in over.items():
+        setattr(cfg, k, v)
+    return cfg
+
+
+@pytest.mark.parametrize("policy,sink,window,chunk,over,ok", [
+    # the slot table holds RC_MAX_SLOTS (256) frames
+    (B.RC_SLIDING, 1, 255, 3, {}, True),
+    (B.RC_SLIDING, 1, 256, 3, {}, False),
+    # chunks of up to RC_MAX_CHUNK_FRAMES (16) frames
+    (B.RC_SLIDING, 0, 16, 16, {}, True),
+    (B.RC_SLIDING, 0, 17, 17, {}, False),
+    # Deep Forcing: sink + tail + budget frames within 256
+    (B.RC_DEEP_FORCING, 1, 245, 3, {"df_budget_tokens": 10 * 16}, True),
+    (B.RC_DEEP_FORCING, 1, 245, 3, {"df_budget_tokens": 11 * 16}, False),
+    # MemRoPE: two memory frames beside sink + window
+    (B.RC_MEMROPE, 1, 253, 3, {"mr_alpha_long": 0.9, "mr_alpha_short": 0.5}, True),
+    (B.RC_MEMROPE, 1, 254, 3, {"mr_alpha_long": 0.9, "mr_alpha_short": 0.5}, False),
+    # Relax Forcing: history + chunk frames within one selection CTA's 64
+    (B.RC_RELAX_FORCING, 1, 6, 3, {"rf_history_frames": 61, "rf_weight": 0.5}, True),
+    (B.RC_RELAX_FORCING, 1, 6, 3, {"rf_history_frames": 62, "rf_weight": 0.5}, False),
+])
+def test_config_limits(policy, sink, window, chunk, over, ok):
+    """Each documented size limit: the largest accepted value passes, one more
+    is rejected with RC_EINVAL before anything is allocated."""
+    cfg = _limit_cfg(policy, sink, window, chunk, **over)
+    if ok:
+        assert B.rc_cache_bytes(cfg) > 0
+        h = B.rc_cache_create(cfg, 0, 0)   # host-only handle: the engine accepts it too
+        B.rc_cache_destroy(h)
+    else:
+        with pytest.raises(B.RcError) as e:
+            B.rc_cache_bytes(cfg)
+        assert e.value.status == B.RC_EINVAL
