@@ -47,7 +47,12 @@ class RollingKVCache:
     device=None creates a host-only handle (integer state only, no GPU).
     """
 
-    def __init__(self, cfg: B.rc_config, device: Optional[torch.device] = torch.device("cuda")):
+    def __init__(self, cfg: B.rc_config, device: Optional[torch.device] = torch.device("cuda"),
+                 mem: Optional[torch.Tensor] = None):
+        """``mem``: optional caller-owned uint8 device tensor of at least
+        rc_cache_bytes(cfg) + 256 bytes to hold the cache (default: allocated
+        here); the cache uses its first 256-byte-aligned rc_cache_bytes(cfg)
+        bytes."""
         self.cfg = cfg
         self.nbytes = B.rc_cache_bytes(cfg)
         self.device = device
@@ -56,7 +61,12 @@ class RollingKVCache:
         if device is not None:
             if not torch.cuda.is_available():
                 raise RuntimeError("a device cache needs CUDA")
-            self.mem = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
+            if mem is None:
+                mem = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
+            elif (mem.dtype != torch.uint8 or not mem.is_contiguous() or mem.device.type != "cuda"
+                  or mem.numel() < self.nbytes + 256):
+                raise ValueError("mem must be a contiguous uint8 CUDA tensor of rc_cache_bytes + 256 bytes")
+            self.mem = mem
             ptr = (self.mem.data_ptr() + 255) // 256 * 256
         self.handle = B.rc_cache_create(cfg, ptr, self.nbytes)
         self._staging = {}

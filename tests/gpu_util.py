@@ -16,6 +16,45 @@ from rcutil import config_for, lib_kept, oracle_df_frames, oracle_kept
 
 TOL_MAX, TOL_MEAN, TOL_LSE = 2e-2, 2e-3, 1e-2
 
+GUARD_BYTES = 4096
+GUARD_BYTE = 0xA5
+
+
+class Guarded:
+    """A device buffer between two guard regions the library must never write.
+
+    ``view(dtype, shape)`` is the usable part; ``intact()`` checks that every
+    byte outside it, the guards and any alignment slack, still holds the
+    pattern. Bounds checks in place of a memory checker."""
+
+    def __init__(self, nbytes: int, device="cuda"):
+        self.nbytes = int(nbytes)
+        self.full = torch.full((GUARD_BYTES + self.nbytes + GUARD_BYTES,), GUARD_BYTE, dtype=torch.uint8,
+                               device=device)
+        self.inner = self.full[GUARD_BYTES:GUARD_BYTES + self.nbytes]
+
+    def view(self, dtype, shape):
+        n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        if n > self.nbytes:
+            raise ValueError("view larger than the buffer")
+        return self.inner[:n].view(dtype).view(shape)
+
+    def intact(self, used: int = None) -> bool:
+        used = self.nbytes if used is None else used
+        lo = self.full[:GUARD_BYTES]
+        hi = self.full[GUARD_BYTES + used:]
+        return bool((lo == GUARD_BYTE).all()) and bool((hi == GUARD_BYTE).all())
+
+
+def guarded_like(shape, dtype, fill=None, device="cuda"):
+    """(buffer, tensor): a guarded tensor of ``shape`` (filled with ``fill``)."""
+    n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+    g = Guarded(n, device)
+    t = g.view(dtype, shape)
+    if fill is not None:
+        t.fill_(fill)
+    return g, t
+
 
 def dev_bf16(bits: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
@@ -83,7 +122,10 @@ class Runner:
         self.layer = layer
         self.seed = seed
         cfg = config_for(w, layers=layers if layers is not None else w.layers)
-        self.cache = RollingKVCache(cfg)
+        # the cache block sits between guard regions, checked after every step
+        self.block = Guarded(B.rc_cache_bytes(cfg) + 256)
+        self.cache = RollingKVCache(cfg, mem=self.block.inner)
+        assert self.block.inner.data_ptr() % 256 == 0
         self.oracle = OracleStream(w, layer=layer, seed=seed)
         self.pairs = (cfg.rope_t_pairs, cfg.rope_h_pairs, cfg.rope_w_pairs)
         if self.pairs == (0, 0, 0):
@@ -105,14 +147,29 @@ class Runner:
             self.oracle.reindex(1 | 2, w.cut_delta)
         q, k, v = rc_synth.chunk_qkv(w, self.layer, chunk, pass_, self.seed)
         Nq = q.shape[0]
-        lse = torch.empty((w.heads, Nq), dtype=torch.float32, device="cuda")
+        # every buffer the call touches sits between guard regions
+        guards = []
+
+        def guarded_input(bits):
+            g, t = guarded_like(bits.shape, torch.bfloat16)
+            t.copy_(dev_bf16(bits))
+            guards.append(g)
+            return t
+        qd, kd, vd = guarded_input(q), guarded_input(k), guarded_input(v)
+        g, lse = guarded_like((w.heads, Nq), torch.float32)
+        guards.append(g)
+        g, out_d = guarded_like(qd.shape, torch.bfloat16)
+        guards.append(g)
         sc = tc = None
         if scores or self.df:
-            sc = torch.full((w.footprint_tokens,), -1.0, dtype=torch.float32, device="cuda")
+            g, sc = guarded_like((w.footprint_tokens,), torch.float32, fill=-1.0)
+            guards.append(g)
         if scores and w.topc:
-            tc = torch.full((w.topc,), -7, dtype=torch.int32, device="cuda")
-        out = self.cache.step(self.layer, dev_bf16(q), dev_bf16(k), dev_bf16(v), chunk * w.chunk_frames,
+            g, tc = guarded_like((w.topc,), torch.int32, fill=-7)
+            guards.append(g)
+        out = self.cache.step(self.layer, qd, kd, vd, chunk * w.chunk_frames, out=out_d,
                               lse=lse, scores=sc, topc=tc, C=w.topc if tc is not None else 0)
+        assert out.data_ptr() == out_d.data_ptr()
         if self.df:
             # the region is chosen from the library's own scores of the last step (DF2)
             kept = self.oracle.step(chunk, pass_, pool_scores=self.prev_scores)
@@ -120,6 +177,12 @@ class Runner:
             kept = self.oracle.step(chunk, pass_)
         torch.cuda.synchronize()
         self.cache.device_status()
+        # nothing written outside the cache block or the output tensors, and
+        # the inputs are left as they were
+        assert self.block.intact(self.cache.nbytes), "write outside the cache block"
+        assert all(g.intact() for g in guards), "write outside an input or output tensor"
+        for dev, bits in ((qd, q), (kd, k), (vd, v)):
+            assert np.array_equal(bits_of(dev), bits.view(np.uint16).reshape(dev.shape)), "input modified"
         st = self.cache.state(self.layer)
         if self.rf:
             kept = self._check_rf_selection(st)
