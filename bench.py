@@ -25,7 +25,6 @@ import datetime
 import hashlib
 import json
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -80,17 +79,38 @@ def kernel_source_hash() -> str:
 
 
 def attention_traffic():
-    """DRAM bytes per attention launch from the committed ncu summary, if it
-    was taken on the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", "attention_wan13b_ncu.md")
+    """DRAM bytes per attention launch (dram__bytes_read.sum +
+    dram__bytes_write.sum of one ncu capture of a steady-state layer-pass),
+    from the machine-readable capture summary, if that capture was taken on
+    the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "attention_wan13b_ncu.json")
     if not os.path.exists(path):
         return None
-    text = open(path).read()
-    sha = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
-    val = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not sha or not val or sha.group(1) != kernel_source_hash():
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("kernel_source_sha256_16") != kernel_source_hash():
         return None
-    return float(val.group(1))
+    return float(rec["dram_bytes_per_launch"])
+
+
+def _find_clock(obj, want_sustained: bool, path=""):
+    """An SM clock (MHz) recorded next to the peaks: the first numeric field
+    whose key path names a clock and (or not) the sustained run."""
+    if isinstance(obj, dict):
+        for k, v in obj.items():
+            r = _find_clock(v, want_sustained, f"{path}/{k}".lower())
+            if r is not None:
+                return r
+        return None
+    if isinstance(obj, (int, float)) and ("mhz" in path or "clock" in path) and "mem" not in path \
+            and "max" not in path and (("sustain" in path) == want_sustained):
+        return float(obj)
+    return None
+
+
+def peak_clock_mhz(peaks, sustained: bool):
+    """SM clock under which the measured GEMM peak was taken, if recorded."""
+    return _find_clock(peaks, sustained)
 
 
 class ClockSampler:
@@ -404,6 +424,31 @@ def run_ours(args, w):
     app = prof["append"]
     app_gbs = (app["bytes"] / max(1, app["launches"])) / (app["ms"] / max(1, app["timed"]) / 1e3) / 1e9
 
+    # the HBM-bound kernels at 40 heads (append, rotate-copy, in-place
+    # re-rotation), each in its own single-layer stream after the timed region
+    hbm = None
+    if rank == 0 and not args.no_hbm:
+        hbm = hbm_cases(dev, steps=10, warmup=2)
+        hbm["append_12_heads"] = {"gbs": app_gbs, "frac": app_gbs / float(peaks.get("hbm_gbs", 6650.0)),
+                                  "ms_per_launch": app["ms"] / max(1, app["timed"]),
+                                  "bytes_per_launch": app["bytes"] / max(1, app["launches"]),
+                                  "note": "inside the timed step above"}
+    if world > 1:
+        dist.barrier()
+
+    # the attention's rate and the GEMM peak at the same SM clock: achieved
+    # per MHz of the sampled median clock over the peak per MHz of the clock
+    # the peak was measured at (when the peaks record it)
+    clk = clocks.summary()
+    peak_mhz = peak_clock_mhz(peaks, sustained=True)
+    burst_mhz = peak_clock_mhz(peaks, sustained=False)
+    sm_mhz = clk.get("sm_mhz")
+
+    def per_clock(pk, mhz):
+        if not mhz or not sm_mhz:
+            return None
+        return (achieved / sm_mhz) / (pk / mhz)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         dt, fl, threads = oracle_sample_seconds(w, heads=3)
@@ -431,12 +476,18 @@ def run_ours(args, w):
                          "kernel": "attention (tcgen05)",
                          "peak_source": f"{peak_src} bf16_tflops_sustained",
                          "frac_of_burst": achieved / float(peaks.get("bf16_tflops", peak)),
+                         "frac_same_clock": per_clock(peak, peak_mhz),
+                         "frac_of_burst_same_clock": per_clock(float(peaks.get("bf16_tflops", peak)), burst_mhz),
+                         "clock_note": (f"attention at a median {sm_mhz} MHz; sustained peak at "
+                                        f"{peak_mhz} MHz, burst peak at {burst_mhz} MHz "
+                                        "(None: not recorded with the peaks)"),
                          "flops_per_launch": att_flops_launch, "ms_per_launch": att_ms},
             "kernels": {k: {"launches": v["launches"], "ms_per_launch": v["ms"] / max(1, v["timed"])}
                         for k, v in prof.items() if v["launches"]},
             "append_gbs": app_gbs, "append_hbm_frac": app_gbs / float(peaks.get("hbm_gbs", 6650.0)),
+            "hbm": hbm,
             "gpu_launches": launches,
-            "clocks": clocks.summary(),
+            "clocks": clk,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
@@ -447,23 +498,23 @@ def run_ours(args, w):
     return 0
 
 
-def run_hbm(args):
+HBM_CASES = ("append", "rotcopy", "inplace")
+
+
+def hbm_cases(dev, steps: int, warmup: int, only=HBM_CASES):
     """HBM-bound kernels at sizes where launch latency does not dominate.
 
     Three single-layer streams with 40 heads x 128 and 1560-token frames, run
     through rc_step; the library's per-launch CUDA events isolate the kernel:
       append    -- fused RoPE + append of a 3-frame chunk (287.5 MB per launch)
       rotcopy   -- Rolling Sink with static sink semantics: every step rotates
-                   the 15 sink frames again from the raw bank (479 MB)
+                   the 15 sink frames again from the raw bank (958 MB)
       inplace   -- sliding window with an 18-frame sink whose time index moves
                    by one every step: in-place time rotation (198 MB)
-    Prints one JSON line with GB/s and the fraction of the measured HBM copy
-    bandwidth for each."""
+    Returns {case: {launches, ms_per_launch, bytes_per_launch, gbs, frac}}."""
     import torch
     from rolling_kv_cache_b200 import binding as B
     from rolling_kv_cache_b200.cache import RollingKVCache
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
     peaks, src = load_peaks()
     hbm = float(peaks.get("hbm_gbs", 6650.0))
     base = rc_synth.WORKLOADS["large"]
@@ -474,7 +525,6 @@ def run_hbm(args):
         "inplace": (base.replace(sink_frames=18, window_frames=3), "rerotate", 1),
     }
     res = {}
-    only = [c for c in args.hbm_cases.split(",") if c] if args.hbm_cases else list(cases)
     for name, (w, kind, sink_shift) in cases.items():
         if name not in only:
             continue
@@ -491,11 +541,11 @@ def run_hbm(args):
             cache.step(0, q, k, v, chunk * w.chunk_frames, out=out)
             chunk += 1
 
-        for _ in range(w.footprint_frames // w.chunk_frames + 1 + args.warmup):
+        for _ in range(w.footprint_frames // w.chunk_frames + 1 + warmup):
             step()
         torch.cuda.synchronize()
-        B.rc_profile_begin(cache.handle, 8 * args.steps + 16)
-        for _ in range(args.steps):
+        B.rc_profile_begin(cache.handle, 8 * steps + 16)
+        for _ in range(steps):
             step()
         torch.cuda.synchronize()
         prof = B.rc_profile_end(cache.handle)[kind]
@@ -506,10 +556,22 @@ def run_hbm(args):
                      "gbs": gbs, "frac": gbs / hbm}
         cache.close()
         del q, k, v, out
+    res["peak_gbs"] = hbm
+    res["peak_source"] = f"{src} hbm_gbs"
+    res["config"] = {"heads": 40, "head_dim": 128, "frame_seqlen": 1560}
+    return res
+
+
+def run_hbm(args):
+    """--hbm: only the HBM-bound kernels (see hbm_cases), one JSON line."""
+    import torch
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    only = [c for c in args.hbm_cases.split(",") if c] if args.hbm_cases else list(HBM_CASES)
+    res = hbm_cases(dev, args.steps, args.warmup, only)
     print(json.dumps({"metric": "HBM GB/s of the append and re-rotation kernels", "unit": "GB/s",
-                      "peak": hbm, "peak_source": f"{src} hbm_gbs", "steps": args.steps,
-                      "config": {"heads": 40, "head_dim": 128, "frame_seqlen": 1560}, **res}),
-          flush=True)
+                      "peak": res.pop("peak_gbs"), "peak_source": res.pop("peak_source"), "steps": args.steps,
+                      "config": res.pop("config"), **res}), flush=True)
     return 0
 
 
@@ -589,11 +651,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="wan13b", choices=list(rc_synth.WORKLOADS))
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--shard", choices=["streams", "heads"], default="streams",
                     help="streams: an independent stream per rank (weak scaling); heads: each rank "
                          "owns a head range of one stream, scores summed over ranks before top-C")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-hbm", action="store_true",
+                    help="skip the HBM-bound kernel cases (40 heads) after the timed region")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (small profiling runs)")
     ap.add_argument("--sdpa-context", action="store_true",

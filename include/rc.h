@@ -238,13 +238,25 @@ rc_status rc_select_topc(void* handle, int layer, const float* scores, int C, in
  * which every GPU that loads the library holds until the process exits. It
  * calls no cudaMalloc, cudaFree or other allocating routine.
  *
- * Arguments, layouts, results and errors are exactly those of rc_step. In
- * addition:
+ * Arguments, layouts and results are those of rc_step. Differences:
+ *   - Only device handles: a host-only handle (dev_mem == NULL) is rejected
+ *     with RC_EINVAL (rc_step accepts it and only advances the state).
  *   - The scratch a call needs is heads * chunk_frames * frame_seqlen *
- *     (head_dim * 2 + 4) bytes plus 8 bytes per cached token, each part
- *     rounded up to 256 bytes; a config needing more than 16 MiB is rejected
- *     with RC_ERANGE before anything is enqueued (e.g. 12 heads x 128 with
- *     4680-token chunks fits; 40 heads does not).
+ *     (head_dim * 2 + 4) bytes (rotated queries and log-sum-exps) plus 8
+ *     bytes per cache row for the two token-score buffers, each part rounded
+ *     up to 256 bytes. The cache rows per head are rc_cache_layout's
+ *     `capacity`: (sink_frames + window_frames) * frame_seqlen, plus
+ *     2 * df_budget_tokens (Deep Forcing) or 2 * rf_history_frames *
+ *     frame_seqlen (Relax Forcing), plus 2 * frame_seqlen (MemRoPE). A config
+ *     needing more than 16 MiB is rejected with RC_ERANGE before anything is
+ *     planned or enqueued (e.g. 12 heads x 128 with 4680-token chunks fits;
+ *     40 heads does not).
+ *   - The attention runs with one CTA per (head, 256-query block) and never
+ *     splits a block between CTAs, so it needs no partial-result rows; with
+ *     more blocks than SMs it runs in several waves.
+ *   - Only the rotated queries, log-sum-exps and token-score buffers move to
+ *     the static array. The device status word and, under Relax Forcing, the
+ *     chunk's frame descriptors stay in the caller's block, as in rc_step.
  *   - The first call on each device looks the array's device address up
  *     (cudaGetSymbolAddress, with that device current) and remembers it; make
  *     that first call before any stream capture.
@@ -252,7 +264,8 @@ rc_status rc_select_topc(void* handle, int layer, const float* scores, int C, in
  *     keeps the last call's contents (whatever must start at zero is cleared
  *     by the call itself). Calls whose work overlaps on the GPU -- different
  *     streams without ordering between them -- race on it: order them.
- *   - The handle's own scratch region in the caller's block is not touched.
+ *   - Errors: those of rc_step, plus RC_EINVAL for a host-only handle and
+ *     RC_ERANGE for a config beyond the static maximum.
  */
 rc_status rc_step_noalloc(void* handle, int layer, const void* q, const void* k_new,
                           const void* v_new, int frame_start, int n_frames, rc_policy policy,

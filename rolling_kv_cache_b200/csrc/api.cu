@@ -219,6 +219,7 @@ struct Cache {
   float* part_o = nullptr;
   float* part_lse = nullptr;
   int sm_count = 148;
+  int dev_id = -1;  // CUDA device ordinal the block was created on (device handles)
   // candidate frames (slot, logical position) of each layer's last step, for rc_select_topc
   std::vector<std::vector<std::pair<int, int>>> last_cand;
   // Deep Forcing per layer: region token sources [2][budget] and the pool selection [budget]
@@ -234,6 +235,21 @@ struct Cache {
 
 rc_status check_handle(const void* h) {
   if (!h) return set_err(RC_EINVAL, "null handle");
+  return RC_OK;
+}
+
+// A device handle's kernels and copies must run on the GPU that holds its
+// memory block: with another device current they would be launched there
+// against memory of another GPU. Checked before anything is planned or
+// enqueued.
+rc_status check_device(const Cache* c) {
+  if (!c->device) return RC_OK;
+  int dev = -1;
+  if (cudaError_t e = cudaGetDevice(&dev)) return cuda_err(e, "cudaGetDevice");
+  if (dev != c->dev_id)
+    return set_err(RC_EINVAL, "the current CUDA device (" + std::to_string(dev) +
+                                  ") is not the device the cache was created on (" +
+                                  std::to_string(c->dev_id) + ")");
   return RC_OK;
 }
 
@@ -318,8 +334,9 @@ rc_status rc_cache_create(const rc_config* cfg, void* dev_mem, size_t bytes, voi
     c->part_lse = reinterpret_cast<float*>(b + m.off_part_lse);
     c->rf_cur = reinterpret_cast<float*>(b + m.off_rf_cur);
     int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+    if (cudaError_t e = cudaGetDevice(&dev)) return cuda_err(e, "cudaGetDevice");
+    c->dev_id = dev;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
       c->sm_count = sms;
     cudaError_t e = cudaMemset(c->mem, 0, m.total);
     if (e != cudaSuccess) return cuda_err(e, "cudaMemset");
@@ -370,6 +387,7 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
   const rc_config& cfg = c->cfg;
   if (policy != cfg.policy) return set_err(RC_EINVAL, "policy differs from the cache's policy");
   if (C < 0 || (C > 0 && !topc) || (topc && C == 0)) return set_err(RC_EINVAL, "topc needs C > 0");
+  if (rc_status st = check_device(c)) return st;
   if (c->device) {
     if (!q || !k_new || !v_new || !out) return set_err(RC_EINVAL, "null tensor");
     for (const void* ptr : {q, k_new, v_new, (const void*)out})
@@ -739,6 +757,7 @@ rc_status rc_select_topc(void* handle, int layer, const float* scores, int C, in
   if (rc_status st = check_handle(handle)) return st;
   Cache* c = static_cast<Cache*>(handle);
   if (!c->device) return set_err(RC_EINVAL, "rc_select_topc needs a device handle");
+  if (rc_status st = check_device(c)) return st;
   if (layer < 0 || layer >= c->cfg.layers) return set_err(RC_EINVAL, "layer out of range");
   if (!scores || !topc || C <= 0) return set_err(RC_EINVAL, "scores, topc and C > 0 are required");
   if ((int)c->last_cand.size() <= layer) return set_err(RC_ESTATE, "no step has run on this layer");
@@ -771,6 +790,7 @@ rc_status rc_step_noalloc(void* handle, int layer, const void* q, const void* k_
   if (rc_status st = check_handle(handle)) return st;
   Cache* c = static_cast<Cache*>(handle);
   if (!c->device) return set_err(RC_EINVAL, "rc_step_noalloc needs a device handle");
+  if (rc_status st = check_device(c)) return st;
   const rc_config& cfg = c->cfg;
   const MemPlan& m = c->mp;
   const size_t q_bytes = align_up((size_t)cfg.heads * m.q_stride * cfg.head_dim * 2);
@@ -850,6 +870,7 @@ rc_status rc_comp_tokens(void* handle, int layer, int32_t* frame, int32_t* tok, 
   if ((c->cfg.policy != RC_DEEP_FORCING && c->cfg.policy != RC_RELAX_FORCING) || !c->device)
     return set_err(RC_EINVAL, "rc_comp_tokens needs a Deep or Relax Forcing device handle");
   if (layer < 0 || layer >= c->cfg.layers) return set_err(RC_EINVAL, "layer out of range");
+  if (rc_status st = check_device(c)) return st;
   const rc::LayerState& L = c->engine->layer(layer);
   if (L.comp_n == 0) return RC_OK;
   if (!frame || !tok) return set_err(RC_EINVAL, "null output array");
@@ -872,6 +893,7 @@ rc_status rc_pool_scores(void* handle, int layer, float* scores, int32_t* n, voi
   if (c->cfg.policy != RC_RELAX_FORCING || !c->device)
     return set_err(RC_EINVAL, "rc_pool_scores needs a Relax Forcing device handle");
   if (layer < 0 || layer >= c->cfg.layers) return set_err(RC_EINVAL, "layer out of range");
+  if (rc_status st = check_device(c)) return st;
   if (!scores || !n) return set_err(RC_EINVAL, "null output");
   std::vector<float> buf(RC_MAX_SLOTS + 1);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -889,6 +911,7 @@ rc_status rc_device_status(void* handle, void* stream) {
   if (rc_status st = check_handle(handle)) return st;
   Cache* c = static_cast<Cache*>(handle);
   if (!c->device) return RC_OK;
+  if (rc_status st = check_device(c)) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaError_t e = cudaStreamSynchronize(s)) return cuda_err(e, "stream sync");
   int word = 0;
@@ -924,6 +947,7 @@ rc_status rc_watchdog_selftest(void* handle, unsigned limit_us, void* stream) {
   if (rc_status st = check_handle(handle)) return st;
   Cache* c = static_cast<Cache*>(handle);
   if (!c->device) return set_err(RC_EINVAL, "host-only handle");
+  if (rc_status st = check_device(c)) return st;
   if (limit_us == 0 || limit_us > 5000000u) return set_err(RC_EINVAL, "limit_us must be in (0, 5e6]");
   if (cudaError_t e = rc::launch_watchdog_selftest(c->status, limit_us, static_cast<cudaStream_t>(stream)))
     return cuda_err(e, "watchdog launch");
@@ -934,6 +958,7 @@ rc_status rc_profile_begin(void* handle, int max_launches) {
   if (rc_status st = check_handle(handle)) return st;
   Cache* c = static_cast<Cache*>(handle);
   if (!c->device) return set_err(RC_EINVAL, "host-only handle");
+  if (rc_status st = check_device(c)) return st;
   if (max_launches < 0 || max_launches > (1 << 20)) return set_err(RC_EINVAL, "max_launches out of range");
   Profiler& p = c->prof;
   p.release();

@@ -580,13 +580,13 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant
 template <int D>
 cudaError_t launch_fwd_d(const AttnParams& p, cudaStream_t s) {
   using L = FwdLayout<D>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)L::kDynSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDevice attr_set;
+  int done = 0;
+  cudaError_t e = attr_set.get(&done, [](int, int* x) {
+    *x = 1;
+    return cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kDynSmem);
+  });
+  if (e != cudaSuccess) return e;
   attn_fwd_kernel<D><<<p.n_ctas, kFwdThreads, L::kDynSmem, s>>>(p);
   return cudaGetLastError();
 }

@@ -3,6 +3,7 @@
 // copy of plans.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -19,6 +20,33 @@ constexpr int kMaxCandFrames = RC_MAX_SLOTS;
 constexpr int kMaxPersistentCtas = 160;
 // Most 256-query pairs a persistent attention launch schedules (per head).
 constexpr int kMaxPairs = 128;
+
+// Values the launchers look up once per device: a kernel's dynamic shared
+// memory attribute (cudaFuncSetAttribute acts on the current device only), the
+// SM count, a grid-stride kernel's resident blocks. One entry per device
+// ordinal, so a process that drives several GPUs gets each device's own
+// value; lock-free, and two threads that race compute the same value.
+constexpr int kMaxDevices = 64;
+struct PerDevice {
+  std::atomic<int> v[kMaxDevices];
+  // *out = the current device's value; `compute(dev, &x)` fills it the first
+  // time (x must come out nonzero).
+  template <typename Fn>
+  cudaError_t get(int* out, Fn compute) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    int x = v[dev].load(std::memory_order_acquire);
+    if (x == 0) {
+      e = compute(dev, &x);
+      if (e != cudaSuccess) return e;
+      v[dev].store(x, std::memory_order_release);
+    }
+    *out = x;
+    return cudaSuccess;
+  }
+};
 
 struct RopeTables {
   const float2* t;  // [t_max][pt]   (cos, sin)

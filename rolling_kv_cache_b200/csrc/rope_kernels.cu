@@ -282,30 +282,22 @@ __global__ void __launch_bounds__(256) mem_update_kernel(const __grid_constant__
   }
 }
 
-int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
-// Blocks of 256 threads of `kernel` resident at once on the GPU. The
-// grid-stride kernels below launch at most one full wave: blocks beyond it
-// would only start when others finish their whole loops and leave the tail of
-// the launch to a few SMs.
+// Blocks of 256 threads of `kernel` resident at once on the current GPU
+// (blocks per SM from the occupancy API x SMs). The grid-stride kernels below
+// launch at most one full wave: blocks beyond it would only start when others
+// finish their whole loops and leave the tail of the launch to a few SMs.
 template <typename Kernel>
-int one_wave(Kernel kernel, int* cache) {
-  if (*cache == 0) {
-    int per_sm = 0;
+int one_wave(Kernel kernel, PerDevice& cache) {
+  int n = 0;
+  const cudaError_t e = cache.get(&n, [kernel](int dev, int* x) {
+    int per_sm = 0, sms = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess || per_sm < 1)
       per_sm = 4;
-    *cache = per_sm * sm_count();
-  }
-  return *cache;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 148;
+    *x = per_sm * sms;
+    return cudaSuccess;
+  });
+  return e == cudaSuccess && n > 0 ? n : 4 * 148;
 }
 
 }  // namespace
@@ -314,9 +306,9 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
   const int rows = p.n_tok * p.H;
   if (rows == 0) return cudaSuccess;
   const dim3 block(p.d / 8, 256 / (p.d / 8));
-  static int wave = 0;
+  static PerDevice wave;
   int blocks = (rows + block.y - 1) / block.y;
-  const int cap = one_wave(append_kernel, &wave);
+  const int cap = one_wave(append_kernel, wave);
   if (blocks > cap) blocks = cap;
   append_kernel<<<blocks, block, 0, s>>>(p);
   return cudaGetLastError();
@@ -327,8 +319,8 @@ cudaError_t launch_rerotate(const RerotateParams& p, cudaStream_t s) {
   const dim3 block(p.d / 8, 256 / (p.d / 8));
   const int rows = p.F * p.H;
   int bx = (rows + block.y - 1) / block.y;
-  static int wave = 0;
-  const int cap = one_wave(rerotate_kernel, &wave) / p.n_jobs;
+  static PerDevice wave;
+  const int cap = one_wave(rerotate_kernel, wave) / p.n_jobs;
   if (bx > cap) bx = cap;
   if (bx < 1) bx = 1;
   rerotate_kernel<<<dim3(bx, p.n_jobs), block, 0, s>>>(p);
@@ -338,9 +330,9 @@ cudaError_t launch_rerotate(const RerotateParams& p, cudaStream_t s) {
 cudaError_t launch_mem_update(const MemUpdateParams& p, cudaStream_t s) {
   const int rows = 2 * p.F * p.H;
   const dim3 block(p.d / 8, 256 / (p.d / 8));
-  static int wave = 0;
+  static PerDevice wave;
   int blocks = (rows + block.y - 1) / block.y;
-  const int cap = one_wave(mem_update_kernel, &wave);
+  const int cap = one_wave(mem_update_kernel, wave);
   if (blocks > cap) blocks = cap;
   mem_update_kernel<<<blocks, block, 0, s>>>(p);
   return cudaGetLastError();
@@ -350,9 +342,9 @@ cudaError_t launch_df_compact(const DfCompactParams& p, cudaStream_t s) {
   const int rows = p.H * p.n_new;
   if (rows == 0) return cudaSuccess;
   const dim3 block(p.d / 8, 256 / (p.d / 8));
-  static int wave = 0;
+  static PerDevice wave;
   int blocks = (rows + block.y - 1) / block.y;
-  const int cap = one_wave(df_compact_kernel, &wave);
+  const int cap = one_wave(df_compact_kernel, wave);
   if (blocks > cap) blocks = cap;
   df_compact_kernel<<<blocks, block, 0, s>>>(p);
   return cudaGetLastError();

@@ -299,13 +299,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const __grid_co
 template <int D>
 cudaError_t launch_scores_d(const ScoreParams& p, cudaStream_t s) {
   using L = ScoreLayout<D>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)L::kDynSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDevice attr_set;
+  int done = 0;
+  cudaError_t e = attr_set.get(&done, [](int, int* x) {
+    *x = 1;
+    return cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kDynSmem);
+  });
+  if (e != cudaSuccess) return e;
   score_kernel<D><<<p.n_ctas, kScoreThreads, L::kDynSmem, s>>>(p);
   return cudaGetLastError();
 }

@@ -12,7 +12,7 @@ from oracle import KeptToken, OracleStream
 from rolling_kv_cache_b200 import binding as B
 from rolling_kv_cache_b200.cache import RollingKVCache
 
-from rcutil import config_for, lib_kept, oracle_df_frames, oracle_kept
+from rcutil import config_for, lib_kept, near_tie_violations, oracle_df_frames, oracle_kept
 
 TOL_MAX, TOL_MEAN, TOL_LSE = 2e-2, 2e-3, 1e-2
 
@@ -139,9 +139,18 @@ class Runner:
         self.mem_state = None     # MemRoPE: fp32 restatement of the device EMA [2 kv][2 mem][F, H, d]
         self.mem_folded = 0
         self.prev_scores = None   # Deep Forcing: the last step's candidate scores (next pool)
+        self.ref_scores = None    # fp64 candidate scores of the current step, when check_float computed them
+        self.df_fp64_checked = 0  # Deep Forcing compactions checked against the fp64 selection
 
-    def step(self, chunk: int, pass_: int, cut: bool = False, scores: bool = False):
+    def step(self, chunk: int, pass_: int, cut: bool = False, scores: bool = False, check: bool = True):
+        """One rc_step of (chunk, pass_) and the oracle's step beside it.
+
+        The integer state is compared on every call. With ``check`` (the
+        default) every buffer the call touches sits between guard regions
+        that are checked afterwards, and the inputs are checked unchanged;
+        ``check=False`` drives the stream quickly to a later event."""
         w = self.w
+        prev_ref, self.ref_scores = self.ref_scores, None
         if cut:
             self.cache.reindex(w.cut_delta, B.RC_REINDEX_FLUSH | B.RC_REINDEX_CUT)
             self.oracle.reindex(1 | 2, w.cut_delta)
@@ -151,22 +160,28 @@ class Runner:
         guards = []
 
         def guarded_input(bits):
+            if not check:
+                return dev_bf16(bits)
             g, t = guarded_like(bits.shape, torch.bfloat16)
             t.copy_(dev_bf16(bits))
             guards.append(g)
             return t
+
+        def guarded_out(shape, dtype, fill=None):
+            if not check:
+                t = torch.empty(shape, dtype=dtype, device="cuda")
+                return t if fill is None else t.fill_(fill)
+            g, t = guarded_like(shape, dtype, fill=fill)
+            guards.append(g)
+            return t
         qd, kd, vd = guarded_input(q), guarded_input(k), guarded_input(v)
-        g, lse = guarded_like((w.heads, Nq), torch.float32)
-        guards.append(g)
-        g, out_d = guarded_like(qd.shape, torch.bfloat16)
-        guards.append(g)
+        lse = guarded_out((w.heads, Nq), torch.float32)
+        out_d = guarded_out(qd.shape, torch.bfloat16)
         sc = tc = None
         if scores or self.df:
-            g, sc = guarded_like((w.footprint_tokens,), torch.float32, fill=-1.0)
-            guards.append(g)
+            sc = guarded_out((w.footprint_tokens,), torch.float32, fill=-1.0)
         if scores and w.topc:
-            g, tc = guarded_like((w.topc,), torch.int32, fill=-7)
-            guards.append(g)
+            tc = guarded_out((w.topc,), torch.int32, fill=-7)
         out = self.cache.step(self.layer, qd, kd, vd, chunk * w.chunk_frames, out=out_d,
                               lse=lse, scores=sc, topc=tc, C=w.topc if tc is not None else 0)
         assert out.data_ptr() == out_d.data_ptr()
@@ -181,8 +196,9 @@ class Runner:
         # the inputs are left as they were
         assert self.block.intact(self.cache.nbytes), "write outside the cache block"
         assert all(g.intact() for g in guards), "write outside an input or output tensor"
-        for dev, bits in ((qd, q), (kd, k), (vd, v)):
-            assert np.array_equal(bits_of(dev), bits.view(np.uint16).reshape(dev.shape)), "input modified"
+        if check:
+            for dev, bits in ((qd, q), (kd, k), (vd, v)):
+                assert np.array_equal(bits_of(dev), bits.view(np.uint16).reshape(dev.shape)), "input modified"
         st = self.cache.state(self.layer)
         if self.rf:
             kept = self._check_rf_selection(st)
@@ -197,6 +213,8 @@ class Runner:
                 frames, toks = self.cache.comp_tokens(self.layer)
                 assert list(zip(frames, toks)) == comp          # the selection, bit-exact
                 assert st.comp_tau0 == self.oracle.df.frame_taus()[1]
+            if self.oracle.df.last_selection is not None and prev_ref is not None:
+                self._check_df_selection_fp64(prev_ref)
             self.prev_scores = sc.cpu().numpy()[:st.n_candidates]
         else:
             assert lib_kept(st) == oracle_kept(kept)
@@ -228,6 +246,23 @@ class Runner:
         want_q = rope_fp32(last["q"], tq, np.tile(hh, w.chunk_frames), np.tile(ww, w.chunk_frames),
                            self.tables, self.pairs)
         assert np.array_equal(qr, want_q)
+
+    def _check_df_selection_fp64(self, ref_scores):
+        """Deep Forcing: the region the device chose at this compaction (equal,
+        bit for bit, to the top-C of the device's own scores of the last pass,
+        which the oracle was fed) against the region the fp64 scores of that
+        pass choose. They may differ only among near-ties: every pool token in
+        the symmetric difference has an fp64 score within SCORE_TOL of the
+        C-th highest fp64 pool score (the same allowance as the top-C of the
+        token scores, reading S1 (ii))."""
+        df = self.oracle.df
+        pool = df.last_pool
+        s64 = np.asarray(ref_scores[:len(pool)], dtype=np.float64)
+        assert len(s64) == len(pool), "fp64 scores do not cover the pool"
+        assert len(df.last_selection) == df.C
+        bad = near_tie_violations(s64, df.last_selection, df.C)
+        assert not bad, ("selection differs from fp64 beyond near-ties", bad[:8])
+        self.df_fp64_checked += 1
 
     def _check_rf_selection(self, st):
         """Relax Forcing: the device's pool scores match fp64 within 1e-4, its
@@ -329,10 +364,16 @@ class Runner:
         assert np.array_equal(got_v, raw_v)
 
     def check_float(self, rows=None, heads=None, scores=False):
+        """O / LSE of the last step against fp64 (sampled rows and heads, or
+        all). With ``scores`` (every row and head) the fp64 candidate scores
+        are kept for the next step: a Deep Forcing compaction there is
+        checked against the selection they make."""
         ref = self.oracle.outputs(heads=heads, rows=rows, want_scores=scores)
         rows = ref["rows"]
         mx, mean, lmx = compare(self.last["out"], self.last["lse"], ref, rows, ref["heads"])
         assert mx <= TOL_MAX and mean <= TOL_MEAN and lmx <= TOL_LSE, (mx, mean, lmx)
+        if scores:
+            self.ref_scores = ref["scores"]
         return ref, (mx, mean, lmx)
 
     def close(self):

@@ -15,6 +15,31 @@ REGION = {0: "sink", 1: "hist", 2: "cur"}
 SCORE_TOL = 2.0 ** -9
 
 
+def near_tie_violations(scores64, got, C: int, tol: float = SCORE_TOL):
+    """Indices where a selection of C candidates differs from the fp64 top-C
+    by more than a near-tie.
+
+    ``scores64`` are the fp64 scores of the candidates (index = position),
+    ``got`` the selected positions. The fp64 selection is the C highest,
+    ties to the lower index (reading S1); a position in the symmetric
+    difference of the two selections is allowed only if its fp64 score lies
+    within ``tol * max(1, kth)`` of the C-th highest fp64 score ``kth``.
+    Returns the offending positions (empty: the selection passes)."""
+    import numpy as np
+    from oracle import top_c
+    s = np.asarray(scores64, dtype=np.float64)
+    got = np.asarray(got, dtype=np.int64)
+    if len(s) <= C:
+        return sorted(set(range(len(s))) ^ set(got.tolist()))
+    want = top_c(s, np.arange(len(s)), C)
+    kth = np.sort(s)[::-1][C - 1]
+    bad = [int(i) for i in set(want.tolist()) ^ set(got.tolist())
+           if not (0 <= i < len(s)) or abs(s[i] - kth) > tol * max(1.0, kth)]
+    if len(set(got.tolist())) != C:
+        bad.append(-1)
+    return sorted(bad)
+
+
 def config_for(w: rc_synth.Workload, **over):
     kw = dict(layers=w.layers, heads=w.heads, head_dim=w.head_dim, grid_h=w.grid_h,
               grid_w=w.grid_w, sink_frames=w.sink_frames, window_frames=w.window_frames,

@@ -17,7 +17,7 @@ from rolling_kv_cache_b200 import binding as B
 from rolling_kv_cache_b200.cache import RollingKVCache
 
 from gpu_util import Runner, bits_of, dev_bf16, rope_fp32, rope_fp32_delta
-from rcutil import SCORE_TOL, config_for
+from rcutil import SCORE_TOL, config_for, near_tie_violations
 
 pytestmark = pytest.mark.gpu
 
@@ -182,13 +182,12 @@ def _topc_checks(w, r, ref):
     assert np.array_equal(got[:n], want)
     assert np.all(got[n:] == -1)
     # (ii) against the fp64 selection, swaps only among near-ties of the C-th score
-    ref_sel = set(ref["topc"].tolist())
-    diff = ref_sel.symmetric_difference(set(want.tolist()))
-    if diff and n < len(cand):
-        kth = np.sort(sr)[::-1][n - 1]
+    if n < len(cand):
         pos = {int(c): i for i, c in enumerate(cand)}
-        for c in diff:
-            assert abs(sr[pos[c]] - kth) <= SCORE_TOL * max(1.0, kth)
+        bad = near_tie_violations(sr, [pos[int(c)] for c in got[:n]], n)
+        assert not bad, bad[:8]
+    else:
+        assert np.array_equal(np.sort(ref["topc"]), got[:n])
 
 
 @pytest.mark.parametrize("d", [128, 64])
@@ -249,6 +248,8 @@ def test_deep_forcing_small():
             assert np.max(np.abs(sg - sr)) <= SCORE_TOL * max(1.0, np.max(np.abs(sr)))
         compacted += r.oracle.df.last_selection is not None
     assert compacted >= 8
+    # every compaction's region also checked against the region fp64 scores choose
+    assert r.df_fp64_checked == compacted
     r.close()
 
 
@@ -257,10 +258,14 @@ def test_deep_forcing_repeat_passes_and_zero_budget():
     w = W["deep_forcing"].replace(heads=2, grid_h=4, grid_w=8, chunks=9, passes=2,
                                   df_budget_tokens=2 * 32)
     r = Runner(w)
+    compacted = 0
     for c, p, g0, cut in rc_synth.stream_schedule(w):
         r.step(c, p)
         r.check_df_region_bitexact()
-        r.check_float()
+        # fp64 scores of the last pass: the next chunk's region is checked against them
+        r.check_float(scores=p == w.passes - 1)
+        compacted += p == 0 and r.oracle.df.last_selection is not None
+    assert compacted >= 3 and r.df_fp64_checked == compacted
     r.close()
     w0 = w.replace(df_budget_tokens=0, passes=1)
     r = Runner(w0)
@@ -330,30 +335,45 @@ def test_memrope_small(alphas):
 SAMPLE_ROWS = np.array([0, 1, 127, 128, 1559, 1560, 1561, 3119, 3120, 4607, 4608, 4679])
 
 
-def _sampled(w, steps, layer=0, layers=None, scores_at=()):
+def _sampled(w, steps, layer=0, layers=None, scores_at=(), fp64_scores_at=()):
+    """Drive a full-size stream through chunk max(steps). At ``steps``: the
+    append bit-exact (first pass) and O / LSE on sampled rows against fp64.
+    At ``scores_at``: the token scores positive with total mass below H Nq,
+    and top-C exact on the kernel's own scores. At ``fp64_scores_at``: O /
+    LSE on every row and head, every token score against fp64 within
+    SCORE_TOL, and the top-C against the fp64 selection up to near-ties.
+    Other chunks run without guard checks, integer state still exact."""
     rng = np.random.default_rng(0)
     rows = np.unique(np.concatenate([SAMPLE_ROWS, rng.integers(0, w.query_tokens, 20)]))
     r = Runner(w, layer=layer, layers=layers)
     last_chunk = max(steps)
+    fp64_checked = 0
     for c, p, g0, cut in rc_synth.stream_schedule(w):
         if c > last_chunk:
             break
-        want_scores = c in scores_at
-        r.step(c, p, cut, scores=want_scores)
+        full = c in fp64_scores_at
+        want_scores = c in scores_at or full
+        r.step(c, p, cut, scores=want_scores, check=c in steps or want_scores)
         if c in steps:
             if p == 0:
                 r.check_append_bitexact()
-            r.check_float(rows=rows)
+            if not full:
+                r.check_float(rows=rows)
             st = r.last["state"]
             assert st.valid_tokens == min(g0 + 3, w.footprint_frames) * w.frame_seqlen or \
                 w.policy == rc_synth.POLICY_INFINITY_ROPE
-        if want_scores:
+        if full:
+            ref, _ = r.check_float(scores=True)
+            _topc_checks(w, r, ref)
+            fp64_checked += 1
+        elif want_scores:
             sg = r.last["scores"]
             want = top_c(sg, np.arange(len(sg)) + 0, w.topc)  # positions; remapped below
             cand_lpos = np.nonzero(np.repeat([e.region == 1 for e in r.last["state"].kept[:r.last["state"].n_kept]],
                                              w.frame_seqlen))[0]
             assert np.array_equal(r.last["topc"], np.sort(cand_lpos[want]))
             assert np.all(sg > 0) and sg.sum() < w.heads * w.query_tokens
+    assert fp64_checked == len(set(fp64_scores_at))
     r.close()
 
 
@@ -367,18 +387,29 @@ def test_full_large_sampled():
 
 
 def test_full_rolling_sink_sampled():
-    _sampled(W["rolling_sink"], steps={0, 5, 6, 7, 8, 12})
+    # through the first roll period (block 12: the bank reversed) and into the
+    # second (blocks 18, 19: the bank forward again, content period 12)
+    _sampled(W["rolling_sink"], steps={0, 5, 6, 7, 8, 12, 18, 19})
 
 
 def test_full_infinity_rope_sampled():
-    w = W["infinity_rope"].replace(cut_chunks=(9, 27, 60))
-    _sampled(w, steps={0, 6, 7, 9, 10}, scores_at={7, 9, 10})
+    """The Infinity-RoPE workload as configured (flush + cut 21 at chunks 27
+    and 60 of the stream): sampled rows around both cuts, token scores and
+    top-C (C = 4680) against fp64 at a steady-state chunk (10: 23400
+    candidates) and right after the first cut (28: 9360 candidates)."""
+    w = W["infinity_rope"]
+    assert w.cut_chunks == (27, 60)
+    _sampled(w, steps={0, 6, 7, 9, 10, 26, 27, 28, 60, 61}, scores_at={7, 9, 27, 60},
+             fp64_scores_at={10, 28})
 
 
 def test_full_deep_forcing_sampled():
     """Full-size Deep Forcing stream (12 heads, 1560-token frames, 3-frame
     deep sink + 18720-token region + 6-frame tail): the region selection
-    exact every step, region keys bit-exact, sampled rows within the bar."""
+    exact every step, region keys bit-exact, sampled rows within the bar; at
+    the steady-state chunk 8 every token score against fp64, and chunk 9's
+    compaction (pool of 23400 tokens, budget 18720) against the region the
+    fp64 scores choose, up to near-ties."""
     w = W["deep_forcing"]
     rng = np.random.default_rng(0)
     rows = np.unique(np.concatenate([SAMPLE_ROWS, rng.integers(0, w.query_tokens, 20)]))
@@ -386,11 +417,19 @@ def test_full_deep_forcing_sampled():
     for c, p, g0, cut in rc_synth.stream_schedule(w):
         if c > 9:
             break
-        r.step(c, p)
-        if c in (0, 3, 4, 8, 9):
+        r.step(c, p, check=c in (0, 3, 4, 8, 9))
+        if c in (0, 3, 4, 9):
             r.check_append_bitexact()
             r.check_df_region_bitexact()
             r.check_float(rows=rows)
+        if c == 8:
+            r.check_append_bitexact()
+            r.check_df_region_bitexact()
+            ref, _ = r.check_float(scores=True)
+            sg, sr = r.last["scores"], ref["scores"]
+            assert len(sg) == len(sr) == w.df_budget_tokens + 3 * w.frame_seqlen
+            assert np.max(np.abs(sg - sr)) <= SCORE_TOL * max(1.0, np.max(np.abs(sr)))
+    assert r.df_fp64_checked == 1
     st = r.last["state"]
     assert st.comp_tokens == w.df_budget_tokens and st.valid_tokens == w.footprint_tokens
     r.close()

@@ -4,19 +4,21 @@ Its per-call scratch lives in the library's static device array instead of
 the caller's block. It is checked here, through the C ABI, against rc_step on
 an identical second cache fed identical inputs, for consecutive calls of a
 stream that uses every scratch region (rotated queries, log-sum-exps, token
-scores and top-C). This file is collected last on purpose.
+scores and top-C); at full size, where its attention grid has more
+(head, query-block) units than the GPU has SMs, against the fp64 oracle.
+This file is collected last on purpose.
 """
 import numpy as np
 import pytest
 import torch
 
 import rc_synth
-from oracle import top_c
+from oracle import OracleStream, top_c
 from rolling_kv_cache_b200 import binding as B
 from rolling_kv_cache_b200.cache import RollingKVCache
 
-from gpu_util import bits_of, dev_bf16, f32
-from rcutil import config_for
+from gpu_util import TOL_LSE, TOL_MAX, TOL_MEAN, bits_of, dev_bf16, f32
+from rcutil import config_for, lib_kept, oracle_kept
 
 pytestmark = pytest.mark.gpu
 
@@ -85,4 +87,41 @@ def test_noalloc_rejects_scratch_beyond_its_maximum():
                           out.data_ptr())
     assert e.value.status == B.RC_ERANGE and "static maximum" in str(e.value)
     assert cache.state(0).frames_committed == 0     # nothing happened
+    cache.close()
+
+
+def test_noalloc_full_size_grid_beyond_sms_against_oracle():
+    # The Infinity-RoPE workload at full size: 12 heads x 128, 4680-query
+    # chunks, 32760 cached tokens, token scores + top-C 4680 every step. Its
+    # step scratch (14.9 MB) fits the static array, and its 12 x 19 = 228
+    # (head, query-block) units exceed the SM count, so the one-CTA-per-unit
+    # grid runs in more than one wave.
+    w = rc_synth.WORKLOADS["infinity_rope"].replace(chunks=9)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert w.heads * ((w.query_tokens + 255) // 256) > sms
+    cache = RollingKVCache(config_for(w))
+    oracle = OracleStream(w)
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([[0, 1, 255, 256, 1559, 1560, 3119, 3120, 4607, 4679],
+                                     rng.integers(0, w.query_tokens, 22)]))
+    checked = 0
+    for c in range(w.chunks):
+        o, lse, sc, tc = _run(cache, B.rc_step_noalloc, w, c, False)
+        kept = oracle.step(c, 0)
+        st = cache.state(0)
+        assert lib_kept(st) == oracle_kept(kept)
+        # top-C exact on the call's own scores (ties to the lower index)
+        lpos = np.nonzero(np.repeat([e.region == 1 for e in st.kept[:st.n_kept]], w.frame_seqlen))[0]
+        n = min(w.topc, len(sc))
+        if n:
+            assert np.array_equal(tc[:n], np.sort(lpos[top_c(sc, np.arange(len(sc)), w.topc)]))
+        assert np.all(tc[n:] == -1)
+        if c in (0, 7, 8):
+            ref = oracle.outputs(rows=rows)
+            err = np.abs(f32(o)[rows].astype(np.float64) - ref["o"])
+            lerr = np.abs(lse[:, rows] - ref["lse"])
+            assert err.max() <= TOL_MAX and err.mean() <= TOL_MEAN and lerr.max() <= TOL_LSE, \
+                (c, err.max(), err.mean(), lerr.max())
+            checked += 1
+    assert checked == 3
     cache.close()
