@@ -93,24 +93,31 @@ def attention_traffic():
     return float(rec["dram_bytes_per_launch"])
 
 
-def _find_clock(obj, want_sustained: bool, path=""):
-    """An SM clock (MHz) recorded next to the peaks: the first numeric field
-    whose key path names a clock and (or not) the sustained run."""
+def _clock_fields(obj, path=""):
+    """(key path, value) of every numeric field under a clock-like key."""
     if isinstance(obj, dict):
+        out = []
         for k, v in obj.items():
-            r = _find_clock(v, want_sustained, f"{path}/{k}".lower())
-            if r is not None:
-                return r
-        return None
-    if isinstance(obj, (int, float)) and ("mhz" in path or "clock" in path) and "mem" not in path \
-            and "max" not in path and (("sustain" in path) == want_sustained):
-        return float(obj)
-    return None
+            out += _clock_fields(v, f"{path}/{k}".lower())
+        return out
+    if isinstance(obj, (int, float)) and not isinstance(obj, bool) and ("mhz" in path or "clock" in path) \
+            and "mem" not in path and "max" not in path and 300 <= obj <= 3000:
+        return [(path, float(obj))]
+    return []
 
 
 def peak_clock_mhz(peaks, sustained: bool):
-    """SM clock under which the measured GEMM peak was taken, if recorded."""
-    return _find_clock(peaks, sustained)
+    """SM clock under which the measured GEMM peak was taken, if the peaks
+    record it: among the clock fields, those naming (or not) the sustained
+    run, preferring ones tied to the bf16 GEMM and to a median."""
+    cands = [(pth, v) for pth, v in _clock_fields(peaks) if ("sustain" in pth) == sustained]
+    if not cands:
+        return None
+
+    def rank(item):
+        pth = item[0]
+        return (-sum(w in pth for w in ("bf16", "gemm", "matmul", "mm", "tflops")), -("median" in pth), pth)
+    return sorted(cands, key=rank)[0][1]
 
 
 class ClockSampler:

@@ -40,10 +40,10 @@ int raw_buffers(const rc_config& c) {
 
 struct MemPlan {
   size_t kv_bytes, raw_bytes, q_bytes, lse_bytes, score_bytes, tab_t, tab_h, tab_w, status_bytes,
-      part_o_bytes, part_lse_bytes, df_meta_bytes, df_sel_bytes, rf_desc_bytes, rf_pool_bytes,
+      part_o_bytes, part_lse_bytes, unit_cnt_bytes, df_meta_bytes, df_sel_bytes, rf_desc_bytes, rf_pool_bytes,
       rf_cur_bytes, mem_bytes;
   size_t off_kv, off_raw, off_q, off_lse, off_score_phys, off_score_logical, off_tab_t, off_tab_h,
-      off_tab_w, off_status, off_part_o, off_part_lse, off_df, off_rf_cur, total;
+      off_tab_w, off_status, off_part_o, off_part_lse, off_unit_cnt, off_df, off_rf_cur, total;
   int pt, ph, pw, cap, raw_frames, q_stride;
 };
 
@@ -72,6 +72,8 @@ MemPlan plan_memory(const rc_config& c, int raw_frames) {
   // stream-K partial rows of the attention: 2 slots per persistent CTA, 256 query rows each
   m.part_o_bytes = align_up((size_t)2 * rc::kMaxPersistentCtas * 256 * c.head_dim * 4);
   m.part_lse_bytes = align_up((size_t)2 * rc::kMaxPersistentCtas * 256 * 4);
+  // arrival counters of the cut units (two query tiles each), zero between launches
+  m.unit_cnt_bytes = align_up((size_t)2 * rc::kMaxPersistentCtas * 4);
   // Deep / Relax Forcing per layer: (frame, token) of both region buffers' tokens, and the selection
   m.df_meta_bytes = align_up((size_t)2 * region * 8);
   m.df_sel_bytes = align_up((size_t)region * 4);
@@ -110,6 +112,8 @@ MemPlan plan_memory(const rc_config& c, int raw_frames) {
   o += m.part_o_bytes;
   m.off_part_lse = o;
   o += m.part_lse_bytes;
+  m.off_unit_cnt = o;
+  o += m.unit_cnt_bytes;
   m.off_df = o;
   o += (m.df_meta_bytes + m.df_sel_bytes + m.rf_desc_bytes + m.rf_pool_bytes + m.mem_bytes) * c.layers;
   m.off_rf_cur = o;
@@ -144,16 +148,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [heads][rows][d] bf16, head stride `head_stride_rows` rows; box {64, 128, 1}, 128B swizzle.
-rc_status make_map(CUtensorMap* map, void* base, int d, int rows, int heads, long long head_stride_rows) {
+// [heads][rows][d] bf16, head stride `head_stride_rows` rows; box {box_x, box_rows, 1}.
+rc_status make_map(CUtensorMap* map, void* base, int d, int rows, int heads, long long head_stride_rows,
+                   int box_x = 64, int box_rows = 128, bool swizzle128 = true) {
   auto fn = encode_fn();
   if (!fn) return set_err(RC_ECUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)heads};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)head_stride_rows * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return set_err(RC_ECUDA, "cuTensorMapEncodeTiled failed: " + std::to_string(r));
   return RC_OK;
@@ -207,6 +212,10 @@ struct Cache {
   MemPlan mp{};
   std::vector<uint16_t*> kc, vc, rawk, rawv;
   std::vector<CUtensorMap> tm_k, tm_v;
+  // K ring boxes of the time-pair chunks for the TMA in-place re-rotation
+  // (empty when the time pairs do not all sit in the first 64 dims)
+  std::vector<CUtensorMap> tm_kt;
+  int ip_ct = 0, ip_rows = 0;
   CUtensorMap tm_q{};
   int tm_q_rows = -1;
   std::vector<float> tab[3];
@@ -218,6 +227,7 @@ struct Cache {
   int* status = nullptr;
   float* part_o = nullptr;
   float* part_lse = nullptr;
+  int* unit_cnt = nullptr;
   int sm_count = 148;
   int dev_id = -1;  // CUDA device ordinal the block was created on (device handles)
   // candidate frames (slot, logical position) of each layer's last step, for rc_select_topc
@@ -332,6 +342,7 @@ rc_status rc_cache_create(const rc_config* cfg, void* dev_mem, size_t bytes, voi
     c->status = reinterpret_cast<int*>(b + m.off_status);
     c->part_o = reinterpret_cast<float*>(b + m.off_part_o);
     c->part_lse = reinterpret_cast<float*>(b + m.off_part_lse);
+    c->unit_cnt = reinterpret_cast<int*>(b + m.off_unit_cnt);
     c->rf_cur = reinterpret_cast<float*>(b + m.off_rf_cur);
     int dev = 0, sms = 0;
     if (cudaError_t e = cudaGetDevice(&dev)) return cuda_err(e, "cudaGetDevice");
@@ -356,6 +367,16 @@ rc_status rc_cache_create(const rc_config* cfg, void* dev_mem, size_t bytes, voi
       const int planes = cfg->heads * (cfg->head_dim / 64);
       if (rc_status st = make_map(&c->tm_k[l], c->kc[l], 64, m.cap, planes, m.cap)) return st;
       if (rc_status st = make_map(&c->tm_v[l], c->vc[l], 64, m.cap, planes, m.cap)) return st;
+    }
+    if (m.pt > 0 && 2 * m.pt <= 64) {
+      c->ip_ct = (2 * m.pt + 7) / 8;
+      c->ip_rows = rc::inplace_box_rows(cfg->frame_seqlen);
+      c->tm_kt.resize(L);
+      const int planes = cfg->heads * (cfg->head_dim / 64);
+      for (int l = 0; l < L; ++l)
+        if (rc_status st = make_map(&c->tm_kt[l], c->kc[l], 64, m.cap, planes, m.cap, 8 * c->ip_ct, c->ip_rows,
+                                    false))
+          return st;
     }
     e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_err(e, "cache init");
@@ -516,8 +537,36 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
     if (cudaError_t e = rc::launch_df_compact(cp, s)) return cuda_err(e, "compact launch");
   }
 
-  // K2: re-rotation jobs (before the append; they touch other slots)
-  for (size_t j0 = 0; j0 < plan.jobs.size(); j0 += rc::kMaxJobs) {
+  // K2: re-rotation jobs (before the append; they touch other slots). In-place
+  // time deltas go to the TMA-staged kernel, rotate-copies to the other; the
+  // jobs of one step target distinct slots.
+  std::vector<const rc::Job*> inplace, rotcopy;
+  for (const rc::Job& jb : plan.jobs) (jb.mode == rc::kInPlace && !c->tm_kt.empty() ? inplace : rotcopy).push_back(&jb);
+  for (size_t j0 = 0; j0 < inplace.size(); j0 += rc::kMaxJobs) {
+    rc::InplaceParams ip;
+    std::memset(&ip, 0, sizeof(ip));
+    ip.tm = c->tm_kt[layer];
+    ip.kc = c->kc[layer];
+    ip.tab_t = c->rt.t;
+    ip.status = c->status;
+    ip.pt = m.pt;
+    ip.ct = c->ip_ct;
+    ip.planes = d / 64;
+    ip.F = F;
+    ip.H = H;
+    ip.cap = m.cap;
+    ip.R = c->ip_rows;
+    ip.tiles_per_head = (F + c->ip_rows - 1) / c->ip_rows;
+    ip.n_jobs = (int)std::min<size_t>(rc::kMaxJobs, inplace.size() - j0);
+    for (int j = 0; j < ip.n_jobs; ++j) {
+      ip.slot[j] = inplace[j0 + j]->dst_slot;
+      ip.delta[j] = inplace[j0 + j]->delta;
+    }
+    // the time pairs of every row read and written: 2 F H (2 pt) x 2 B per job
+    Timed tm(c->prof, RC_KERNEL_REROTATE, s, 0.0, (double)ip.n_jobs * F * H * 2 * (2 * m.pt) * 2);
+    if (cudaError_t e = rc::launch_rerotate_inplace(ip, s)) return cuda_err(e, "in-place rerotate launch");
+  }
+  for (size_t j0 = 0; j0 < rotcopy.size(); j0 += rc::kMaxJobs) {
     rc::RerotateParams rp{};
     rp.kc = c->kc[layer];
     rp.vc = c->vc[layer];
@@ -528,9 +577,9 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
     rp.F = F;
     rp.cap = m.cap;
     rp.raw_cap = m.raw_frames * F;
-    rp.n_jobs = (int)std::min<size_t>(rc::kMaxJobs, plan.jobs.size() - j0);
+    rp.n_jobs = (int)std::min<size_t>(rc::kMaxJobs, rotcopy.size() - j0);
     for (int j = 0; j < rp.n_jobs; ++j) {
-      const rc::Job& jb = plan.jobs[j0 + j];
+      const rc::Job& jb = *rotcopy[j0 + j];
       rp.job[j] = rc::RerotateJob{jb.dst_slot, jb.mode, jb.src_frame, jb.sigma, jb.delta, jb.copy_v};
     }
     rp.rt = c->rt;
@@ -622,6 +671,7 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
     const bool split = c->part_o != nullptr && units > G && NP <= rc::kMaxPairs;
     at.part_o = split ? c->part_o : nullptr;
     at.part_lse = split ? c->part_lse : nullptr;
+    at.unit_cnt = split ? c->unit_cnt : nullptr;
     at.n_ctas = split ? G : units;
     if (split) {
       // stream-K ranges that level the work: CTA c ran round units c, c + G, ...;
@@ -675,10 +725,6 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
     {
       Timed tm(c->prof, RC_KERNEL_ATTENTION, s, 4.0 * d * H * pairs, 0.0);
       if (cudaError_t e = rc::launch_attention(at, d, s)) return cuda_err(e, "attention launch");
-    }
-    if (at.part_o && (at.n_pairs * H) % at.n_ctas != 0) {
-      Timed tm(c->prof, RC_KERNEL_COMBINE, s, 0.0, (double)2 * at.n_ctas * 256 * (d + 1) * 4);
-      if (cudaError_t e = rc::launch_attention_combine(at, d, s)) return cuda_err(e, "combine launch");
     }
   }
 
@@ -918,6 +964,8 @@ rc_status rc_device_status(void* handle, void* stream) {
   if (cudaError_t e = cudaMemcpy(&word, c->status, 4, cudaMemcpyDeviceToHost)) return cuda_err(e, "status read");
   if (word) {
     cudaMemset(c->status, 0, 4);
+    // a kernel that gave up may have left cut units counted but not merged
+    cudaMemset(c->unit_cnt, 0, c->mp.unit_cnt_bytes);
     return set_err(RC_ETIMEOUT, "a device-side wait gave up (status word " + std::to_string(word) + ")");
   }
   return RC_OK;

@@ -95,6 +95,22 @@ struct RerotateParams {
   RopeTables rt;
 };
 
+// K2 in place, staged by TMA: R_t(delta_j) composed onto the time pairs of
+// every key row of slot slot[j], for each job j. The tensor map covers the
+// K ring [H * d/64][cap][64] with a box of the first 8 ct dims (the 16-byte
+// chunks that hold time pairs) x R rows of one plane-0 row block.
+struct InplaceParams {
+  CUtensorMap tm;      // K ring as (64, cap, H * d/64), box {8 ct, R, 1}, no swizzle
+  uint16_t* kc;
+  const float2* tab_t; // time table [t_max][pt] (cos, sin)
+  int* status;
+  int pt, ct, planes, F, H, cap, R;
+  int tiles_per_head;  // ceil(F / R)
+  int n_jobs;
+  int slot[kMaxJobs];
+  int delta[kMaxJobs];
+};
+
 struct KvSegment {
   int tok_start;
   int len;
@@ -111,6 +127,7 @@ struct alignas(64) AttnParams {
   int* status;         // device status word
   float* part_o;       // null, or stream-K partials [2 * n_ctas][256][d] fp32 (O / l)
   float* part_lse;     // [2 * n_ctas][256] fp32, log2-sum-exp of each partial row
+  int* unit_cnt;       // [2 * kMaxPersistentCtas] arrivals per (cut unit, query tile); 0 between launches
   int n_ctas;          // grid size: persistent CTAs (with partials) or one per (head, pair)
   int Nq, H, F, mask_block;
   float scale_log2;    // log2(e) / sqrt(d)
@@ -151,9 +168,10 @@ struct TopCParams {
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t launch_rerotate(const RerotateParams& p, cudaStream_t s);
+cudaError_t launch_rerotate_inplace(const InplaceParams& p, cudaStream_t s);
+// Rows per TMA box of the in-place kernel for frames of F tokens.
+int inplace_box_rows(int F);
 cudaError_t launch_attention(const AttnParams& p, int head_dim, cudaStream_t s);
-// K5: merges the partial rows of split (head, pair) units; only after a launch with partials.
-cudaError_t launch_attention_combine(const AttnParams& p, int head_dim, cudaStream_t s);
 cudaError_t launch_scores(const ScoreParams& p, int head_dim, cudaStream_t s);
 cudaError_t launch_topc(const TopCParams& p, cudaStream_t s);
 cudaError_t launch_watchdog_selftest(int* status, unsigned limit_us, cudaStream_t s);

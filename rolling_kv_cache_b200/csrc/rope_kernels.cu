@@ -15,8 +15,11 @@
 // restatement reproduces it bit for bit.
 #include "kernels.cuh"
 #include "df_compact.cuh"
+#include "ptx.cuh"
 
 #include <cuda_bf16.h>
+
+#include <algorithm>
 
 namespace rc {
 
@@ -165,6 +168,104 @@ __global__ void __launch_bounds__(256) rerotate_kernel(const __grid_constant__ R
       if (jb.copy_v)
         *reinterpret_cast<uint4*>(p.vc + dst) = __ldg(reinterpret_cast<const uint4*>(p.raw_v + src));
     }
+  }
+}
+
+// K2 in place, TMA-staged. The time pairs of a key row are its first 2 pt
+// dims, which sit in plane 0: ct 16-byte chunks (96 of the row's 128 bytes
+// at pt = 22). Each work item is one (job, head, block of R rows) of a slot;
+// a TMA box brings the item's R x 8 ct dims into a ring of kStages
+// shared-memory stages, so every CTA keeps kStages boxes of reads in flight
+// instead of one 16-byte load per thread. Threads rotate their chunks from
+// shared memory and store them back with 16-byte stores, only the rows of
+// the slot (a box past the slot's last row reads rows it never writes).
+// Thread t always handles chunk t % ct of a row, so its four (cos, sin)
+// pairs are loaded once per item. Bounded waits; on give-up the CTA waits
+// (bounded) for its loads in flight and returns with RC_ETIMEOUT recorded.
+constexpr int kInplaceStages = 4;
+
+__global__ void __launch_bounds__(256) rerotate_inplace_kernel(const __grid_constant__ InplaceParams p) {
+  extern __shared__ __align__(128) uint8_t ip_smem[];
+  __shared__ uint64_t full[kInplaceStages];
+  __shared__ int abort_sh;
+  const int tid = threadIdx.x;
+  const int stage_bytes = (p.R * p.ct * 16 + 127) & ~127;
+  const int n_items = p.n_jobs * p.H * p.tiles_per_head;
+  const int G = gridDim.x;
+  const int n_local = blockIdx.x < n_items ? (n_items - blockIdx.x + G - 1) / G : 0;
+  if (tid == 0) {
+    for (int s = 0; s < kInplaceStages; ++s) ptx::mbar_init(&full[s], 1);
+    abort_sh = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  volatile int* abort = &abort_sh;
+  auto issue = [&](int i) {  // local item i into stage i % kInplaceStages (thread 0)
+    const int item = blockIdx.x + i * G;
+    const int j = item / (p.H * p.tiles_per_head);
+    const int rem = item - j * p.H * p.tiles_per_head;
+    const int h = rem / p.tiles_per_head;
+    const int b = rem - h * p.tiles_per_head;
+    uint64_t* bar = &full[i % kInplaceStages];
+    ptx::mbar_arrive_expect_tx(bar, (uint32_t)(p.R * p.ct * 16));
+    ptx::tma_load_3d(&p.tm, bar, ip_smem + (i % kInplaceStages) * stage_bytes, 0, p.slot[j] * p.F + b * p.R,
+                     h * p.planes);
+  };
+  if (tid == 0) {
+    ptx::fence_proxy_async_smem();
+    for (int i = 0; i < n_local && i < kInplaceStages; ++i) issue(i);
+  }
+  const int c8 = tid % p.ct;
+  const int row_step = blockDim.x / p.ct;
+  const bool active = tid < row_step * p.ct;
+  int i = 0;
+  for (; i < n_local; ++i) {
+    const int st = i % kInplaceStages;
+    const bool ok = ptx::mbar_wait(&full[st], (i / kInplaceStages) & 1, abort, p.status, RC_ETIMEOUT);
+    if (ok && active) {
+      const int item = blockIdx.x + i * G;
+      const int j = item / (p.H * p.tiles_per_head);
+      const int rem = item - j * p.H * p.tiles_per_head;
+      const int h = rem / p.tiles_per_head;
+      const int b = rem - h * p.tiles_per_head;
+      const int r0 = b * p.R;
+      const int nrows = min(p.R, p.F - r0);
+      const int delta = p.delta[j];
+      const float sgn = delta < 0 ? -1.f : 1.f;
+      const int adelta = delta < 0 ? -delta : delta;
+      float cs_c[4], cs_s[4];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int m = c8 * 4 + jj;
+        const float2 cs = m < p.pt ? __ldg(p.tab_t + (size_t)adelta * p.pt + m) : make_float2(1.f, 0.f);
+        cs_c[jj] = cs.x;
+        cs_s[jj] = sgn * cs.y;
+      }
+      const uint4* src = reinterpret_cast<const uint4*>(ip_smem + st * stage_bytes);
+      uint16_t* dst0 = p.kc + cache_off(h, p.planes, p.cap, p.slot[j] * p.F + r0, c8);
+      for (int row = tid / p.ct; row < nrows; row += row_step) {
+        float f[8];
+        unpack8(src[row * p.ct + c8], f);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+          if (c8 * 4 + jj < p.pt) rot(f[2 * jj], f[2 * jj + 1], cs_c[jj], cs_s[jj]);
+        *reinterpret_cast<uint4*>(dst0 + (size_t)row * 64) = pack8(f);
+      }
+    }
+    // every thread reaches this barrier (the waits are bounded): stage st is
+    // consumed, and all leave together if any wait gave up
+    if (__syncthreads_or(!ok)) break;
+    if (tid == 0 && i + kInplaceStages < n_local) {
+      ptx::fence_proxy_async_smem();
+      issue(i + kInplaceStages);
+    }
+  }
+  if (i < n_local && tid == 0) {
+    // gave up: wait (bounded, ignoring the abort flag) for the loads still in flight
+    int dummy = 0;
+    volatile int* noabort = reinterpret_cast<volatile int*>(&dummy);
+    for (int k = i; k < n_local && k < i + kInplaceStages; ++k)
+      ptx::mbar_wait(&full[k % kInplaceStages], (k / kInplaceStages) & 1, noabort, p.status, RC_ETIMEOUT);
   }
 }
 
@@ -324,6 +425,44 @@ cudaError_t launch_rerotate(const RerotateParams& p, cudaStream_t s) {
   if (bx > cap) bx = cap;
   if (bx < 1) bx = 1;
   rerotate_kernel<<<dim3(bx, p.n_jobs), block, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+int inplace_box_rows(int F) {
+  if (F <= 256) return F;
+  for (int r = 128; r >= 64; --r)
+    if (F % r == 0) return r;
+  return 128;
+}
+
+cudaError_t launch_rerotate_inplace(const InplaceParams& p, cudaStream_t s) {
+  const int n_items = p.n_jobs * p.H * p.tiles_per_head;
+  if (n_items == 0) return cudaSuccess;
+  const int threads = 32 * p.ct;
+  const int smem = kInplaceStages * ((p.R * p.ct * 16 + 127) & ~127);
+  static PerDevice attr_set;
+  static PerDevice wave;
+  int done = 0;
+  cudaError_t e = attr_set.get(&done, [](int, int* x) {
+    *x = 1;
+    return cudaFuncSetAttribute(rerotate_inplace_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
+  });
+  if (e != cudaSuccess) return e;
+  int cap = 0;
+  e = wave.get(&cap, [](int dev, int* x) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 148;
+    *x = sms;
+    return cudaSuccess;
+  });
+  if (e != cudaSuccess) return e;
+  // a few CTAs per SM: each keeps kInplaceStages boxes in flight
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rerotate_inplace_kernel, threads, smem) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const int blocks = std::min(n_items, cap * std::min(per_sm, 4));
+  rerotate_inplace_kernel<<<blocks, threads, smem, s>>>(p);
   return cudaGetLastError();
 }
 

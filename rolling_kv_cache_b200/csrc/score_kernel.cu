@@ -86,10 +86,12 @@ struct ScoreScheduler {
 // 2^x on the FMA pipe, for the share of the exponentials the exp2 unit
 // (16 per clock per SM, the binding pipe of this kernel) should not take:
 // x = n + f with n the nearest integer (added to the exponent bits) and
-// 2^f on [-1/2, 1/2] by a quartic whose coefficients were fitted to the
-// relative error of 2^f at Chebyshev nodes (max relative error 2.7e-6 in
-// fp32). x is clamped at -126, so -inf (a query past the chunk) gives at
-// most 2^-126 instead of 0.
+// 2^f on [-1/2, 1/2] by a quartic: the minimax fit of the relative error of
+// 2^f (Remez exchange in fp64, degree 4, equioscillating error 2.59e-6),
+// each coefficient rounded to fp32 (max relative error 2.7e-6 in fp32
+// arithmetic; tests/test_kernel_math.py re-derives the coefficients and
+// checks the bound). x is clamped at -126, so -inf (a query past the chunk)
+// gives at most 2^-126 instead of 0.
 __device__ __forceinline__ float exp2_fma(float x) {
   x = fmaxf(x, -126.f);
   const float t = __fadd_rn(x, 12582912.f);  // 1.5 * 2^23: round(x) lands in the low mantissa bits

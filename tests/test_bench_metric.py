@@ -42,3 +42,32 @@ def test_wan13b_layer_pass_closed_form():
     assert pairs == F * F * 54
     assert bench.attention_flops(w, n_hist) == 4.0 * d * H * pairs
     assert abs(bench.attention_flops(w, n_hist) / 1e12 - 0.8074) < 1e-4
+
+
+def test_peak_clock_lookup():
+    # the clock the GEMM peak was measured at, found wherever the peaks record it
+    pk = {"hbm_gbs": 6557.8, "bf16_tflops": 1663.7, "bf16_tflops_sustained": 1390.4,
+          "clocks": {"bf16_sustained": {"sm_mhz_median": 1342, "sm_mhz_max": 1965},
+                     "bf16": {"sm_mhz_median": 1890}, "hbm_copy": {"sm_mhz_median": 1965, "mem_mhz": 3996}}}
+    assert bench.peak_clock_mhz(pk, sustained=True) == 1342.0
+    assert bench.peak_clock_mhz(pk, sustained=False) == 1890.0
+    assert bench.peak_clock_mhz({"bf16_tflops": 1663.7}, sustained=True) is None
+
+
+def test_traffic_needs_a_capture_of_the_current_source(tmp_path, monkeypatch):
+    # the roofline's traffic is read from a capture summary only when that
+    # capture was taken on the current attention kernel source
+    import json
+    import os
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.attention_traffic() is None
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "abc")
+    (prof / "attention_wan13b_ncu.json").write_text(json.dumps(
+        {"kernel_source_sha256_16": "abc", "dram_bytes_per_launch": 2.5e8}))
+    assert bench.attention_traffic() == 2.5e8
+    (prof / "attention_wan13b_ncu.json").write_text(json.dumps(
+        {"kernel_source_sha256_16": "old", "dram_bytes_per_launch": 2.5e8}))
+    assert bench.attention_traffic() is None
+    assert os.path.isdir(prof)

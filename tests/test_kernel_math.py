@@ -5,7 +5,9 @@ The score pass computes one exponential in eight on the FMA pipe
 quartic for 2^f on [-1/2, 1/2]. This test reads the quartic's coefficients
 from the kernel source and evaluates the same steps in fp32 (each Horner
 step rounded once, as a fused multiply-add rounds) against the exact 2^x:
-the relative error stays within the bound the kernel's comment states.
+the relative error stays within the bound the kernel's comment states. It
+also re-derives the coefficients: they are the minimax fit of the relative
+error (Remez exchange, degree 4 on [-1/2, 1/2], in fp64), rounded to fp32.
 """
 import os
 import re
@@ -63,3 +65,41 @@ def test_exp2_fma_integers_and_clamp():
     # the probabilities the pass sums
     tiny = _exp2_fma(np.array([-np.inf, -1000.0, -127.5], dtype=np.float32)).astype(np.float64)
     assert np.all((tiny >= 0.0) & (tiny <= 2.0 ** -125))
+
+
+def _remez_relative(deg=4, lo=-0.5, hi=0.5, iters=40):
+    """Minimax polynomial of degree `deg` for 2^f on [lo, hi] in relative
+    error, by the Remez exchange algorithm: start from the Chebyshev
+    extrema, solve p(x_i) / 2^x_i - 1 = (-1)^i E on deg + 2 reference
+    points, move the points to the extrema of the new error, repeat until
+    the reference stops moving. Returns (coefficients lowest first, |E|)."""
+    n = deg + 2
+    x = (lo + hi) / 2 - (hi - lo) / 2 * np.cos(np.pi * np.arange(n) / (n - 1))
+    grid = np.linspace(lo, hi, 200001)
+    for _ in range(iters):
+        A = np.zeros((n, n))
+        for i in range(n):
+            A[i, :deg + 1] = x[i] ** np.arange(deg + 1) / np.exp2(x[i])
+            A[i, deg + 1] = -(-1.0) ** i
+        sol = np.linalg.solve(A, np.ones(n))
+        c, E = sol[:deg + 1], sol[deg + 1]
+        e = np.polyval(c[::-1], grid) / np.exp2(grid) - 1.0
+        cuts = np.concatenate([[0], np.nonzero(np.diff(np.sign(e)))[0] + 1, [len(grid)]])
+        ext = np.array([a + np.argmax(np.abs(e[a:b])) for a, b in zip(cuts[:-1], cuts[1:])])
+        if len(ext) != n:
+            break
+        x_new = grid[ext]
+        if np.allclose(x_new, x, atol=1e-9):
+            break
+        x = x_new
+    return c, abs(E)
+
+
+def test_exp2_fma_coefficients_are_the_minimax_fit():
+    c, E = _remez_relative()
+    assert 2.5e-6 < E < 2.7e-6              # the equioscillating relative error of the degree-4 fit
+    src = np.array(_coefficients()[::-1], dtype=np.float32)   # lowest degree first
+    fit = c.astype(np.float32)
+    # each coefficient is the fp64 minimax coefficient rounded to fp32 (within one fp32 ulp)
+    ulp = np.spacing(np.abs(fit))
+    assert np.all(np.abs(src.astype(np.float64) - fit.astype(np.float64)) <= ulp), (src, fit)
