@@ -363,13 +363,12 @@ rc_status rc_watchdog_selftest(void* handle, unsigned limit_us, void* stream);
 
 /* Per-kernel timing with CUDA events recorded on the launching stream
  * around every kernel a step enqueues (re-rotation, append, attention,
- * scores, top-C, compaction). rc_profile_begin arms it for up to
- * max_launches launches (events are created here, not in rc_step);
- * rc_profile_end synchronizes the recorded events and reports, per kernel
- * kind, the launch count and the summed device milliseconds, then disarms.
- * Launches beyond the limit are counted but not timed. RC_KERNEL_COMBINE
- * counts no launches: the partial rows of attention units split between
- * CTAs are merged inside the attention kernel. */
+ * scores, top-C, compaction, and the merge of attention units split between
+ * CTAs). rc_profile_begin arms it for up to max_launches launches (events
+ * are created here, not in rc_step); rc_profile_end synchronizes the
+ * recorded events and reports, per kernel kind, the launch count and the
+ * summed device milliseconds, then disarms. Launches beyond the limit are
+ * counted but not timed. */
 enum { RC_KERNEL_REROTATE = 0, RC_KERNEL_APPEND = 1, RC_KERNEL_ATTENTION = 2,
        RC_KERNEL_SCORES = 3, RC_KERNEL_TOPC = 4, RC_KERNEL_COMBINE = 5, RC_KERNEL_COMPACT = 6,
        RC_KERNEL_KINDS = 7 };

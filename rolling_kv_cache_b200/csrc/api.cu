@@ -40,10 +40,10 @@ int raw_buffers(const rc_config& c) {
 
 struct MemPlan {
   size_t kv_bytes, raw_bytes, q_bytes, lse_bytes, score_bytes, tab_t, tab_h, tab_w, status_bytes,
-      part_o_bytes, part_lse_bytes, unit_cnt_bytes, df_meta_bytes, df_sel_bytes, rf_desc_bytes, rf_pool_bytes,
+      part_o_bytes, part_lse_bytes, df_meta_bytes, df_sel_bytes, rf_desc_bytes, rf_pool_bytes,
       rf_cur_bytes, mem_bytes;
   size_t off_kv, off_raw, off_q, off_lse, off_score_phys, off_score_logical, off_tab_t, off_tab_h,
-      off_tab_w, off_status, off_part_o, off_part_lse, off_unit_cnt, off_df, off_rf_cur, total;
+      off_tab_w, off_status, off_part_o, off_part_lse, off_df, off_rf_cur, total;
   int pt, ph, pw, cap, raw_frames, q_stride;
 };
 
@@ -72,8 +72,6 @@ MemPlan plan_memory(const rc_config& c, int raw_frames) {
   // stream-K partial rows of the attention: 2 slots per persistent CTA, 256 query rows each
   m.part_o_bytes = align_up((size_t)2 * rc::kMaxPersistentCtas * 256 * c.head_dim * 4);
   m.part_lse_bytes = align_up((size_t)2 * rc::kMaxPersistentCtas * 256 * 4);
-  // arrival counters of the cut units (two query tiles each), zero between launches
-  m.unit_cnt_bytes = align_up((size_t)2 * rc::kMaxPersistentCtas * 4);
   // Deep / Relax Forcing per layer: (frame, token) of both region buffers' tokens, and the selection
   m.df_meta_bytes = align_up((size_t)2 * region * 8);
   m.df_sel_bytes = align_up((size_t)region * 4);
@@ -112,8 +110,6 @@ MemPlan plan_memory(const rc_config& c, int raw_frames) {
   o += m.part_o_bytes;
   m.off_part_lse = o;
   o += m.part_lse_bytes;
-  m.off_unit_cnt = o;
-  o += m.unit_cnt_bytes;
   m.off_df = o;
   o += (m.df_meta_bytes + m.df_sel_bytes + m.rf_desc_bytes + m.rf_pool_bytes + m.mem_bytes) * c.layers;
   m.off_rf_cur = o;
@@ -227,7 +223,6 @@ struct Cache {
   int* status = nullptr;
   float* part_o = nullptr;
   float* part_lse = nullptr;
-  int* unit_cnt = nullptr;
   int sm_count = 148;
   int dev_id = -1;  // CUDA device ordinal the block was created on (device handles)
   // candidate frames (slot, logical position) of each layer's last step, for rc_select_topc
@@ -342,7 +337,6 @@ rc_status rc_cache_create(const rc_config* cfg, void* dev_mem, size_t bytes, voi
     c->status = reinterpret_cast<int*>(b + m.off_status);
     c->part_o = reinterpret_cast<float*>(b + m.off_part_o);
     c->part_lse = reinterpret_cast<float*>(b + m.off_part_lse);
-    c->unit_cnt = reinterpret_cast<int*>(b + m.off_unit_cnt);
     c->rf_cur = reinterpret_cast<float*>(b + m.off_rf_cur);
     int dev = 0, sms = 0;
     if (cudaError_t e = cudaGetDevice(&dev)) return cuda_err(e, "cudaGetDevice");
@@ -671,7 +665,6 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
     const bool split = c->part_o != nullptr && units > G && NP <= rc::kMaxPairs;
     at.part_o = split ? c->part_o : nullptr;
     at.part_lse = split ? c->part_lse : nullptr;
-    at.unit_cnt = split ? c->unit_cnt : nullptr;
     at.n_ctas = split ? G : units;
     if (split) {
       // stream-K ranges that level the work: CTA c ran round units c, c + G, ...;
@@ -725,6 +718,10 @@ rc_status rc_step(void* handle, int layer, const void* q, const void* k_new, con
     {
       Timed tm(c->prof, RC_KERNEL_ATTENTION, s, 4.0 * d * H * pairs, 0.0);
       if (cudaError_t e = rc::launch_attention(at, d, s)) return cuda_err(e, "attention launch");
+    }
+    if (at.part_o && (at.n_pairs * H) % at.n_ctas != 0) {
+      Timed tm(c->prof, RC_KERNEL_COMBINE, s, 0.0, (double)2 * at.n_ctas * 256 * (d + 1) * 4);
+      if (cudaError_t e = rc::launch_attention_combine(at, d, s)) return cuda_err(e, "combine launch");
     }
   }
 
@@ -964,8 +961,6 @@ rc_status rc_device_status(void* handle, void* stream) {
   if (cudaError_t e = cudaMemcpy(&word, c->status, 4, cudaMemcpyDeviceToHost)) return cuda_err(e, "status read");
   if (word) {
     cudaMemset(c->status, 0, 4);
-    // a kernel that gave up may have left cut units counted but not merged
-    cudaMemset(c->unit_cnt, 0, c->mp.unit_cnt_bytes);
     return set_err(RC_ETIMEOUT, "a device-side wait gave up (status word " + std::to_string(word) + ")");
   }
   return RC_OK;

@@ -61,8 +61,7 @@ struct FwdLayout {
 // One unit of work: query pair (rows q0 .. q0+255) of head h over the KV
 // tiles [kv_lo, kv_hi) of the pair's tile walk. slot >= 0: the job covers
 // part of its pair's tiles and leaves (O / l, log2-sum-exp) in the partial
-// workspace, merged by the CTA that writes the unit's last part; slot < 0:
-// it writes the output.
+// workspace for the combine kernel; slot < 0: it writes the output.
 struct Job {
   int h, q0, kv_lo, kv_hi, slot, rq_hi;
   bool has1;
@@ -82,7 +81,7 @@ __device__ __forceinline__ int pair_rq_hi(const AttnParams& p, int pair) {
 // tile) order, are split into G ranges, one per CTA, sized by the host so
 // that every CTA's round tiles plus range tiles come out equal (units differ
 // in length under the in-chunk mask); a unit cut between CTAs leaves partial
-// rows, merged by whichever CTA finishes its last part. Their K/V spans only a few heads, so it stays
+// rows for the combine kernel. Their K/V spans only a few heads, so it stays
 // in L2 whatever the offsets.
 // Without a partial workspace the grid has one CTA per unit.
 struct Scheduler {
@@ -144,91 +143,6 @@ struct Scheduler {
   }
 };
 
-// The CTA whose stream-K range holds tile position pos: the largest c with
-// sk_start[c] <= pos (empty ranges before it share its start).
-__device__ __forceinline__ int owner_of(const AttnParams& p, int G, long long pos) {
-  int lo = 0, hi = G - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (p.sk_start[mid] <= pos) lo = mid;
-    else hi = mid - 1;
-  }
-  return lo;
-}
-
-// The parts of a stream-K unit cut between CTAs: CTAs [c_lo, c_hi] whose
-// ranges are not empty each hold one, in partial slot 2 c (the CTA's first
-// range job: its range starts inside the unit) or 2 c + 1 (its last).
-struct UnitParts {
-  int c_lo, c_hi, n;
-  long long C_u;
-  __device__ UnitParts(const AttnParams& p, int G, int h, int pair) {
-    const int NP = p.n_pairs;
-    const long long u = (long long)h * NP + pair;
-    C_u = (u / NP) * p.pair_prefix[NP] + p.pair_prefix[pair];
-    const int T_u = p.pair_prefix[pair + 1] - p.pair_prefix[pair];
-    c_lo = owner_of(p, G, C_u);
-    c_hi = owner_of(p, G, C_u + T_u - 1);
-    n = 0;
-    for (int cc = c_lo; cc <= c_hi; ++cc) n += has(p, cc);
-  }
-  __device__ static bool has(const AttnParams& p, int cc) { return p.sk_start[cc + 1] > p.sk_start[cc]; }
-  __device__ int slot(const AttnParams& p, int cc) const { return 2 * cc + ((p.sk_start[cc] >= C_u) ? 0 : 1); }
-};
-
-// Merges the parts of one query row of a cut unit into the output:
-// O = sum_i 2^(lse_i - lse) O_i with lse = log2 sum_i 2^(lse_i), for the
-// D/2 columns [col0, col0 + D/2) (and the row's LSE when write_lse). The
-// parts were written by other CTAs: read through L2.
-template <int D>
-__device__ __forceinline__ void merge_row(const AttnParams& p, const UnitParts& up, int prow, int qtok, int h,
-                                          int col0, bool write_lse) {
-  float mx = -INFINITY;
-  for (int cc = up.c_lo; cc <= up.c_hi; ++cc)
-    if (UnitParts::has(p, cc)) mx = fmaxf(mx, __ldcg(p.part_lse + (size_t)up.slot(p, cc) * 2 * kTileRows + prow));
-  float den = 0.f;
-  for (int cc = up.c_lo; cc <= up.c_hi; ++cc)
-    if (UnitParts::has(p, cc)) {
-      const float ls = __ldcg(p.part_lse + (size_t)up.slot(p, cc) * 2 * kTileRows + prow);
-      den += ls == -INFINITY ? 0.f : exp2f(ls - mx);
-    }
-  const float inv = den > 0.f ? 1.f / den : 0.f;
-#pragma unroll
-  for (int cb = 0; cb < D / 2; cb += 32) {
-    float acc[32];
-#pragma unroll
-    for (int k = 0; k < 32; ++k) acc[k] = 0.f;
-    for (int cc = up.c_lo; cc <= up.c_hi; ++cc) {
-      if (!UnitParts::has(p, cc)) continue;
-      const int sl = up.slot(p, cc);
-      const float ls = __ldcg(p.part_lse + (size_t)sl * 2 * kTileRows + prow);
-      const float w = ls == -INFINITY ? 0.f : exp2f(ls - mx);
-      const float4* src =
-          reinterpret_cast<const float4*>(p.part_o + ((size_t)sl * 2 * kTileRows + prow) * D + col0 + cb);
-#pragma unroll
-      for (int v = 0; v < 8; ++v) {
-        const float4 x = __ldcg(src + v);
-        acc[4 * v] += w * x.x;
-        acc[4 * v + 1] += w * x.y;
-        acc[4 * v + 2] += w * x.z;
-        acc[4 * v + 3] += w * x.w;
-      }
-    }
-    uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)qtok * p.H + h) * D + col0 + cb);
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      uint4 x;
-      x.x = ptx::pack_bf16x2(acc[8 * v] * inv, acc[8 * v + 1] * inv);
-      x.y = ptx::pack_bf16x2(acc[8 * v + 2] * inv, acc[8 * v + 3] * inv);
-      x.z = ptx::pack_bf16x2(acc[8 * v + 4] * inv, acc[8 * v + 5] * inv);
-      x.w = ptx::pack_bf16x2(acc[8 * v + 6] * inv, acc[8 * v + 7] * inv);
-      dst[v] = x;
-    }
-  }
-  if (write_lse && p.lse)
-    p.lse[(size_t)h * p.Nq + qtok] = (den > 0.f ? mx + log2f(den) : -INFINITY) * 0.69314718055994531f;
-}
-
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
   using L = FwdLayout<D>;
@@ -238,7 +152,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   __shared__ float swap_buf[2][2][2][kTileRows];  // [group][exchange parity][column half][row]
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
-  __shared__ int merge_sh[2];  // per query tile: this CTA wrote the last part of the cut unit
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t base_u32 = (ptx::smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -424,10 +337,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       other = buf[ch ^ 1][row];
       return true;
     };
-    // Every warp of a group runs every job of the schedule and leaves the loop
-    // only at the group-wide decision at the end of a job, so the group's
-    // named barriers always see all of its 256 threads.
     while (sc.next(jb)) {
+      if (*abort) break;
       if (grp == 1 && !jb.has1) continue;
       const int qtok = jb.q0 + grp * kTileRows + row;
       const int my_rank = (min(qtok, p.Nq - 1) / p.F) / p.mask_block;
@@ -526,11 +437,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       float l_other = 0.f;
       if (ok && !swap(l, l_other)) ok = false;
       const float lt = l + l_other;
-      bool have_o = false;
-      if (ok && done > 0) {
-        have_o = ptx::mbar_wait(&bar_o[grp], (gs - 1) & 1, abort, p.status, RC_ETIMEOUT);
-        ok = have_o;
-      }
+      const bool have_o =
+          ok && done > 0 && ptx::mbar_wait(&bar_o[grp], (gs - 1) & 1, abort, p.status, RC_ETIMEOUT);
       ptx::tc_fence_after();
       const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
       const float lse2 = lt > 0.f ? m * c + __log2f(lt) : -INFINITY;
@@ -573,31 +481,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           p.part_lse[(size_t)jb.slot * 2 * kTileRows + prow] = lse2;
         }
       }
-      // A unit cut between CTAs: the query tile's group that writes the unit's
-      // last part merges all parts into the output. Each writer makes its part
-      // visible device-wide before the count; the counter goes back to 0 for
-      // the next launch. A group in which any wait gave up neither counts nor
-      // merges, and leaves the loop (every thread of the group together).
-      if (jb.slot >= 0) __threadfence();
-      const bool bad = ptx::named_bar_or(1 + grp, 256, !ok);
-      if (jb.slot >= 0 && !bad) {
-        const UnitParts up(p, gridDim.x, jb.h, jb.q0 / (2 * kTileRows));
-        if ((warp & 7) == 0 && lane == 0) {
-          const long long U = (long long)p.n_pairs * p.H;
-          const long long first_rem = (U / gridDim.x) * gridDim.x;
-          const long long u = (long long)jb.h * p.n_pairs + jb.q0 / (2 * kTileRows);
-          int* cnt = p.unit_cnt + 2 * (u - first_rem) + grp;
-          const int last = atomicAdd(cnt, 1) == up.n - 1;
-          if (last) atomicExch(cnt, 0);
-          merge_sh[grp] = last;
-        }
-        ptx::named_bar_sync(1 + grp, 256);
-        if (merge_sh[grp]) {
-          __threadfence();
-          if (qtok < p.Nq) merge_row<D>(p, up, prow, qtok, jb.h, ch * (D / 2), ch == 0);
-        }
-      }
-      if (bad) break;
+      if (!ok) break;
     }
   }
   ptx::tc_fence_before();
@@ -606,6 +490,87 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, 512);
   }
+}
+
+// K5: merges the partial results of the (head, pair) units the stream-K
+// schedule split between CTAs: O = sum_i 2^(lse_i - lse) O_i with
+// lse = log2 sum_i 2^(lse_i). Block (unit, y) takes 32 query rows of the
+// unit; 8 consecutive threads share a row, D/8 columns each, so every warp
+// reads 4 whole rows of a partial at once.
+// The CTA whose stream-K range holds tile position pos: the largest c with
+// sk_start[c] <= pos (empty ranges before it share its start).
+__device__ __forceinline__ int owner_of(const AttnParams& p, int G, long long pos) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.sk_start[mid] <= pos) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+constexpr int kCombineRowsPerBlock = 32;
+
+template <int D>
+__global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant__ AttnParams p, int G) {
+  constexpr int kCols = D / 8;
+  const int NP = p.n_pairs;
+  const long long T_head = p.pair_prefix[NP];
+  const long long U = (long long)NP * p.H;
+  const long long first_rem = (U / G) * G;  // units before it ran in whole-unit rounds
+  const long long u = first_rem + blockIdx.x;
+  if (u >= U) return;
+  const int h = (int)(u / NP), pair = (int)(u % NP);
+  auto cum = [&](long long v) { return (v / NP) * T_head + p.pair_prefix[v % NP]; };
+  const long long C_u = cum(u);  // unit start (tile position)
+  const int T_u = p.pair_prefix[pair + 1] - p.pair_prefix[pair];
+  const int c_lo = owner_of(p, G, C_u), c_hi = owner_of(p, G, C_u + T_u - 1);
+  if (c_lo == c_hi) return;  // written directly by one CTA
+  const int prow = blockIdx.y * kCombineRowsPerBlock + (threadIdx.x >> 3);
+  const int col0 = (threadIdx.x & 7) * kCols;
+  const int qtok = pair * 2 * kTileRows + prow;
+  if (qtok >= p.Nq) return;
+  // slot of CTA c's job on this unit: its first job iff its range starts inside the unit
+  auto slot_of = [&](int cc) { return 2 * cc + ((p.sk_start[cc] >= C_u) ? 0 : 1); };
+  // a CTA whose stream-K range is empty holds no part
+  auto has_part = [&](int cc) { return p.sk_start[cc + 1] > p.sk_start[cc]; };
+  float mx = -INFINITY;
+  for (int cc = c_lo; cc <= c_hi; ++cc)
+    if (has_part(cc)) mx = fmaxf(mx, p.part_lse[(size_t)slot_of(cc) * 2 * kTileRows + prow]);
+  float acc[kCols];
+#pragma unroll
+  for (int k = 0; k < kCols; ++k) acc[k] = 0.f;
+  float den = 0.f;
+  for (int cc = c_lo; cc <= c_hi; ++cc) {
+    if (!has_part(cc)) continue;
+    const int sl = slot_of(cc);
+    const float ls = p.part_lse[(size_t)sl * 2 * kTileRows + prow];
+    const float w = ls == -INFINITY ? 0.f : exp2f(ls - mx);
+    den += w;
+    const float4* src =
+        reinterpret_cast<const float4*>(p.part_o + ((size_t)sl * 2 * kTileRows + prow) * D + col0);
+#pragma unroll
+    for (int v = 0; v < kCols / 4; ++v) {
+      const float4 x = src[v];
+      acc[4 * v] += w * x.x;
+      acc[4 * v + 1] += w * x.y;
+      acc[4 * v + 2] += w * x.z;
+      acc[4 * v + 3] += w * x.w;
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)qtok * p.H + h) * D + col0);
+#pragma unroll
+  for (int v = 0; v < kCols / 8; ++v) {
+    uint4 x;
+    x.x = ptx::pack_bf16x2(acc[8 * v] * inv, acc[8 * v + 1] * inv);
+    x.y = ptx::pack_bf16x2(acc[8 * v + 2] * inv, acc[8 * v + 3] * inv);
+    x.z = ptx::pack_bf16x2(acc[8 * v + 4] * inv, acc[8 * v + 5] * inv);
+    x.w = ptx::pack_bf16x2(acc[8 * v + 6] * inv, acc[8 * v + 7] * inv);
+    dst[v] = x;
+  }
+  if (p.lse && (threadIdx.x & 7) == 0)
+    p.lse[(size_t)h * p.Nq + qtok] = (den > 0.f ? mx + log2f(den) : -INFINITY) * 0.69314718055994531f;
 }
 
 template <int D>
@@ -627,6 +592,19 @@ cudaError_t launch_fwd_d(const AttnParams& p, cudaStream_t s) {
 cudaError_t launch_attention(const AttnParams& p, int head_dim, cudaStream_t s) {
   if (p.Nq <= 0 || p.n_ctas <= 0) return cudaSuccess;
   return head_dim == 64 ? launch_fwd_d<64>(p, s) : launch_fwd_d<128>(p, s);
+}
+
+cudaError_t launch_attention_combine(const AttnParams& p, int head_dim, cudaStream_t s) {
+  if (p.Nq <= 0 || !p.part_o) return cudaSuccess;
+  const int units = p.n_pairs * p.H;
+  const int rem = units % p.n_ctas;  // units of the stream-K remainder
+  if (rem == 0) return cudaSuccess;
+  const dim3 grid(rem, 2 * kTileRows / kCombineRowsPerBlock);
+  if (head_dim == 64)
+    attn_combine_kernel<64><<<grid, 256, 0, s>>>(p, p.n_ctas);
+  else
+    attn_combine_kernel<128><<<grid, 256, 0, s>>>(p, p.n_ctas);
+  return cudaGetLastError();
 }
 
 }  // namespace rc

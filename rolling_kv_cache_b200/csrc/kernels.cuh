@@ -127,7 +127,6 @@ struct alignas(64) AttnParams {
   int* status;         // device status word
   float* part_o;       // null, or stream-K partials [2 * n_ctas][256][d] fp32 (O / l)
   float* part_lse;     // [2 * n_ctas][256] fp32, log2-sum-exp of each partial row
-  int* unit_cnt;       // [2 * kMaxPersistentCtas] arrivals per (cut unit, query tile); 0 between launches
   int n_ctas;          // grid size: persistent CTAs (with partials) or one per (head, pair)
   int Nq, H, F, mask_block;
   float scale_log2;    // log2(e) / sqrt(d)
@@ -172,6 +171,8 @@ cudaError_t launch_rerotate_inplace(const InplaceParams& p, cudaStream_t s);
 // Rows per TMA box of the in-place kernel for frames of F tokens.
 int inplace_box_rows(int F);
 cudaError_t launch_attention(const AttnParams& p, int head_dim, cudaStream_t s);
+// K5: merges the partial rows of split (head, pair) units; only after a launch with partials.
+cudaError_t launch_attention_combine(const AttnParams& p, int head_dim, cudaStream_t s);
 cudaError_t launch_scores(const ScoreParams& p, int head_dim, cudaStream_t s);
 cudaError_t launch_topc(const TopCParams& p, cudaStream_t s);
 cudaError_t launch_watchdog_selftest(int* status, unsigned limit_us, cudaStream_t s);

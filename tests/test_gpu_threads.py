@@ -6,9 +6,8 @@ The launchers keep per-device, thread-safe lookups (kernel attributes, SM
 counts, resident blocks per kernel), and every error message is per thread,
 so two threads each driving their own cache on their own stream must get
 exactly the bytes a single thread gets. The stream-K attention path (more
-(head, query-block) units than SMs, partial rows merged by the CTA that
-writes a cut unit's last part, through arrival counters in each cache's own
-block) is the one exercised.
+(head, query-block) units than SMs, partial rows merged by the combine
+kernel) is the one exercised.
 """
 import threading
 
