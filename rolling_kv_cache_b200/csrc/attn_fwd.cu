@@ -251,14 +251,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       }
       ptx::mma_commit(&bar_s[i]);
     };
-    auto issue_pv = [&](int i, int st, bool acc) {
+    // O_i += P_i V; the commit that tells the epilogue O_i is final goes only
+    // after a job's last PV (a softmax that rescales O at tile j has already
+    // waited for S_i(j), issued after PV_i(j-1), and tcgen05 work completes in
+    // issue order). Each commit costs the issuing thread about 46 cycles,
+    // during which the tensor pipe, fed one MMA at a time, has nothing queued.
+    auto issue_pv = [&](int i, int st, bool acc, bool last) {
       const uint32_t sV = base_u32 + L::kV + st * L::kTile;
       // P of keys [16 ks, 16 ks + 16): column (ks / 4) * 64 + (ks % 4) * 8 of S_i
 #pragma unroll
       for (int ks = 0; ks < kTileRows / 16; ++ks)
         ptx::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + (ks >> 2) * 64 + (ks & 3) * 8,
                     ptx::sdesc_sw128(sV + ks * 2048, kSubTileBytes, 1024), idesc_o, acc || ks > 0);
-      ptx::mma_commit(&bar_o[i]);
+      if (last) ptx::mma_commit(&bar_o[i]);
     };
     int nq = 0, g = 0, gp[2] = {0, 0};
     bool ok = true;
@@ -279,7 +284,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         if (!ptx::mbar_wait(&bar_p[0], gp[0] & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
         if (!ptx::mbar_wait(&bar_vf[st], (g >> 1) & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
         ptx::tc_fence_after();
-        issue_pv(0, st, j > 0);
+        issue_pv(0, st, j > 0, !more);
         ++gp[0];
         if (!two) ptx::mma_commit(&bar_ve[st]);
         if (more) {
@@ -294,7 +299,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         if (two) {
           if (!ptx::mbar_wait(&bar_p[1], gp[1] & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
           ptx::tc_fence_after();
-          issue_pv(1, st, j > 0);
+          issue_pv(1, st, j > 0, !more);
           ++gp[1];
           ptx::mma_commit(&bar_ve[st]);
           if (more) {
@@ -325,7 +330,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     uint64_t* pbar = &bar_pair[grp * 4 + wq];
     const float c = p.scale_log2;
     const float thresh = kRescaleLog2 / c;
-    int gs = 0;  // this group's tiles so far (phase of bar_s / bar_p / bar_o)
+    int gs = 0;  // this group's tiles so far (phase of bar_s / bar_p)
+    int nj = 0;  // this group's jobs so far (phase of bar_o: one commit per job)
     int nx = 0;  // partner exchanges so far (phase of pbar, slot of swap_buf)
     // writes v, returns the partner's value (bounded wait)
     auto swap = [&](float v, float& other) -> bool {
@@ -375,8 +381,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         const bool need = m_new > m + thresh;       // also true for the first visible tile
         const bool real = need && m != -INFINITY;   // O already holds weighted values
         if (__any_sync(0xffffffffu, real)) {
-          if (!ptx::mbar_wait(&bar_o[grp], (gs - 1) & 1, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
-          ptx::tc_fence_after();
+          // PV of the previous tile is complete: it was issued before this
+          // tile's S, which the wait above saw complete
           const float alpha = real ? ptx::ex2((m - m_new) * c) : 1.f;
 #pragma unroll
           for (int cc = 0; cc < D / 64; ++cc) {
@@ -438,7 +444,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       if (ok && !swap(l, l_other)) ok = false;
       const float lt = l + l_other;
       const bool have_o =
-          ok && done > 0 && ptx::mbar_wait(&bar_o[grp], (gs - 1) & 1, abort, p.status, RC_ETIMEOUT);
+          ok && done > 0 && ptx::mbar_wait(&bar_o[grp], nj & 1, abort, p.status, RC_ETIMEOUT);
+      if (done > 0) ++nj;
       ptx::tc_fence_after();
       const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
       const float lse2 = lt > 0.f ? m * c + __log2f(lt) : -INFINITY;
