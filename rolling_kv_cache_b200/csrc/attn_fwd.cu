@@ -41,6 +41,31 @@ namespace rc {
 
 namespace {
 
+// 2^x for a pair of lanes on the FMA pipe, in packed f32x2 steps: n =
+// round(x) by the 1.5 * 2^23 shift, f = x - n in [-1/2, 1/2], 2^f by a cubic,
+// n added to the exponent field. The cubic's coefficients are the minimax fit
+// of the relative error on [-1/2, 1/2] (Remez exchange in fp64, each rounded
+// to fp32): relative error within 7.5e-5, below the 2^-9 of the bf16 P it
+// feeds. x is clamped at -126 so the exponent field cannot wrap; below that
+// the result is at most 2^-126, as the SFU's flush-to-zero gives 0.
+__device__ __forceinline__ float2 exp2_cubic2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = ptx::fadd2(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = ptx::fadd2(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = ptx::ffma2(n, make_float2(-1.f, -1.f), x);
+  float2 q = ptx::ffma2(make_float2(5.517166853e-02f, 5.517166853e-02f), f,
+                        make_float2(2.426111251e-01f, 2.426111251e-01f));
+  q = ptx::ffma2(q, f, make_float2(6.932609677e-01f, 6.932609677e-01f));
+  q = ptx::ffma2(q, f, make_float2(9.999280572e-01f, 9.999280572e-01f));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+// pairs k of a 16-pair chunk with (k % 8) < kCubicPairs take exp2_cubic2;
+// the rest the SFU's ex2 (16 per clock per SM, the bound of the exponential
+// phase when it runs alone)
+constexpr int kCubicPairs = 2;
+
 constexpr int kSoftmaxWarps = 16;
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
@@ -404,13 +429,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         auto emit = [&](const uint32_t (&r)[32], int k0) {
           uint32_t pk[16];
           if (lim_h >= 64) {
+            const float2 c2 = make_float2(c, c), nmc2 = make_float2(-mc, -mc);
+            float2 s2 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-              const float a = ptx::ex2(fmaf(__uint_as_float(r[2 * k]), c, -mc));
-              const float b = ptx::ex2(fmaf(__uint_as_float(r[2 * k + 1]), c, -mc));
-              sum += a + b;
-              pk[k] = ptx::pack_bf16x2(a, b);
+              const float2 x =
+                  ptx::ffma2(make_float2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), c2, nmc2);
+              float2 e;
+              if ((k & 7) < kCubicPairs) {
+                e = exp2_cubic2(x);
+              } else {
+                e.x = ptx::ex2(x.x);
+                e.y = ptx::ex2(x.y);
+              }
+              s2 = ptx::fadd2(s2, e);
+              pk[k] = ptx::pack_bf16x2(e.x, e.y);
             }
+            sum += s2.x + s2.y;
           } else {
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
@@ -471,7 +506,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
             u.y = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
             u.z = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
             u.w = ptx::pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
-            dst[v] = u;
+            __stcs(dst + v, u);  // streamed: leaves L2 before the next launch has to evict it
           }
         } else {
           float4* dst = reinterpret_cast<float4*>(p.part_o + ((size_t)jb.slot * 2 * kTileRows + prow) * D + col);
@@ -565,6 +600,14 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant
       acc[4 * v + 3] += w * x.w;
     }
   }
+  // the partial rows are dead once merged: drop their L2 lines (each 128-byte
+  // line by the first of the threads that read it) instead of letting them
+  // be written back to HBM during a later launch. The lanes still here are
+  // whole 8-lane row groups (a row past Nq left as a group), converged.
+  __syncwarp(__activemask());
+  if ((col0 & 31) == 0)
+    for (int cc = c_lo; cc <= c_hi; ++cc)
+      if (has_part(cc)) ptx::discard_l2(p.part_o + ((size_t)slot_of(cc) * 2 * kTileRows + prow) * D + col0);
   const float inv = den > 0.f ? 1.f / den : 0.f;
   uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)qtok * p.H + h) * D + col0);
 #pragma unroll
@@ -574,7 +617,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __grid_constant
     x.y = ptx::pack_bf16x2(acc[8 * v + 2] * inv, acc[8 * v + 3] * inv);
     x.z = ptx::pack_bf16x2(acc[8 * v + 4] * inv, acc[8 * v + 5] * inv);
     x.w = ptx::pack_bf16x2(acc[8 * v + 6] * inv, acc[8 * v + 7] * inv);
-    dst[v] = x;
+    __stcs(dst + v, x);
   }
   if (p.lse && (threadIdx.x & 7) == 0)
     p.lse[(size_t)h * p.Nq + qtok] = (den > 0.f ? mx + log2f(den) : -INFINITY) * 0.69314718055994531f;

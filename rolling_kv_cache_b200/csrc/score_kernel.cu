@@ -83,44 +83,60 @@ struct ScoreScheduler {
   }
 };
 
-// 2^x on the FMA pipe, for the share of the exponentials the exp2 unit
-// (16 per clock per SM, the binding pipe of this kernel) should not take:
-// x = n + f with n the nearest integer (added to the exponent bits) and
-// 2^f on [-1/2, 1/2] by a quartic: the minimax fit of the relative error of
-// 2^f (Remez exchange in fp64, degree 4, equioscillating error 2.59e-6),
+// 2^x for a pair of lanes on the FMA pipe, for the share of the exponentials
+// the exp2 unit (16 per clock per SM, the binding pipe of this kernel) should
+// not take: x = n + f with n the nearest integer (added to the exponent bits)
+// and 2^f on [-1/2, 1/2] by a quartic: the minimax fit of the relative error
+// of 2^f (Remez exchange in fp64, degree 4, equioscillating error 2.59e-6),
 // each coefficient rounded to fp32 (max relative error 2.7e-6 in fp32
 // arithmetic; tests/test_kernel_math.py re-derives the coefficients and
-// checks the bound). x is clamped at -126, so -inf (a query past the chunk)
-// gives at most 2^-126 instead of 0.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = __fadd_rn(x, 12582912.f);  // 1.5 * 2^23: round(x) lands in the low mantissa bits
-  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
-  float p = 0.009570101276040077f;
-  p = fmaf(p, f, 0.05591785907745361f);
-  p = fmaf(p, f, 0.240247443318367f);
-  p = fmaf(p, f, 0.6931217908859253f);
-  p = fmaf(p, f, 0.9999992847442627f);
-  const uint32_t n = static_cast<uint32_t>(__float_as_int(t) - 0x4B400000);
-  return __uint_as_float(__float_as_uint(p) + (n << 23));
+// checks the bound). Every step is a packed f32x2 instruction: as scalar
+// code the nine dependent steps stall the few warps a sub-partition holds.
+// x is clamped at -126, so -inf (a query past the chunk) gives at most
+// 2^-126 instead of 0.
+__device__ __forceinline__ float2 exp2_quartic2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = ptx::fadd2(x, make_float2(12582912.f, 12582912.f));  // 1.5 * 2^23: round(x) in the low bits
+  const float2 n = ptx::fadd2(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = ptx::ffma2(n, make_float2(-1.f, -1.f), x);
+  float2 q = ptx::ffma2(make_float2(0.009570101276040077f, 0.009570101276040077f), f,
+                        make_float2(0.05591785907745361f, 0.05591785907745361f));
+  q = ptx::ffma2(q, f, make_float2(0.240247443318367f, 0.240247443318367f));
+  q = ptx::ffma2(q, f, make_float2(0.6931217908859253f, 0.6931217908859253f));
+  q = ptx::ffma2(q, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
 // Sum over 32 queries of exp2(s c - lse2): r holds S^T columns (queries)
-// q .. q + 31 of this thread's key, lse the matching lse2 values. One
-// exponential in eight runs on the FMA pipe (measured on B200: one in eight
-// takes 3 % off the pass, one in four gains nothing).
-__device__ __forceinline__ float exp_sum32(const uint32_t (&r)[32], const float* lse, float c) {
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+// q .. q + 31 of this thread's key, nlse the matching -lse2 values. The scale
+// and the sums are packed f32x2 instructions; two pairs in eight take
+// exp2_quartic2 (measured on B200: the exponential phase alone 20 % shorter
+// than with the exp2 unit only, where one scalar exponential in eight on the
+// FMA pipe gained 6 %).
+__device__ __forceinline__ float exp_sum32(const uint32_t (&r)[32], const float* nlse, float c) {
+  const float2 c2 = make_float2(c, c);
+  float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int k = 0; k < 32; k += 4) {
-    const float4 l = *reinterpret_cast<const float4*>(lse + k);
-    a0 += ptx::ex2(fmaf(__uint_as_float(r[k + 0]), c, -l.x));
-    a1 += ptx::ex2(fmaf(__uint_as_float(r[k + 1]), c, -l.y));
-    a2 += ptx::ex2(fmaf(__uint_as_float(r[k + 2]), c, -l.z));
-    if (k & 4) a3 += exp2_fma(fmaf(__uint_as_float(r[k + 3]), c, -l.w));
-    else a3 += ptx::ex2(fmaf(__uint_as_float(r[k + 3]), c, -l.w));
+    const float4 l = *reinterpret_cast<const float4*>(nlse + k);
+    const float2 x0 = ptx::ffma2(make_float2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), c2,
+                                 make_float2(l.x, l.y));
+    const float2 x1 = ptx::ffma2(make_float2(__uint_as_float(r[k + 2]), __uint_as_float(r[k + 3])), c2,
+                                 make_float2(l.z, l.w));
+    float2 e0, e1;
+    if ((k & 15) == 0) {  // pairs 8 i and 8 i + 1 of every eight
+      e0 = exp2_quartic2(x0);
+      e1 = exp2_quartic2(x1);
+    } else {
+      e0 = make_float2(ptx::ex2(x0.x), ptx::ex2(x0.y));
+      e1 = make_float2(ptx::ex2(x1.x), ptx::ex2(x1.y));
+    }
+    a0 = ptx::fadd2(a0, e0);
+    a1 = ptx::fadd2(a1, e1);
   }
-  return (a0 + a1) + (a2 + a3);
+  return (a0.x + a0.y) + (a1.x + a1.y);
 }
 
 template <int D>
@@ -129,7 +145,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const __grid_co
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_q, bar_qe, bar_kf[kKStages], bar_ke[kKStages], bar_s[2][2], bar_sfree[2][2],
       bar_lse[2], bar_fin[2];
-  __shared__ __align__(16) float s_lse[2][2][kTileRows];  // [job parity][query tile][query]
+  __shared__ __align__(16) float s_lse[2][2][kTileRows];  // -lse2: [job parity][query tile][query]
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -253,11 +269,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_kernel(const __grid_co
     bool ok = true;
     while (ok && sc.next(jb)) {
       if (*abort) break;
-      // this job's lse2, written by the first column half (one query each)
+      // this job's -lse2, written by the first column half (one query each)
       float* lse = s_lse[nj & 1][grp];
       if (ch == 0) {
         const int qtok = jb.q0 + grp * kTileRows + key;
-        lse[key] = qtok < p.Nq ? p.lse[(size_t)jb.h * p.Nq + qtok] * 1.4426950408889634f : INFINITY;
+        lse[key] = qtok < p.Nq ? -(p.lse[(size_t)jb.h * p.Nq + qtok] * 1.4426950408889634f) : -INFINITY;
       }
       ptx::mbar_arrive(&bar_lse[grp]);
       if (!ptx::mbar_wait(&bar_lse[grp], nj & 1, abort, p.status, RC_ETIMEOUT)) break;

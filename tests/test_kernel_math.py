@@ -1,13 +1,18 @@
 """Host checks of the arithmetic the kernels hard-code.
 
-The score pass computes one exponential in eight on the FMA pipe
-(`exp2_fma` in score_kernel.cu): 2^x = 2^n 2^f with n = round(x) and a
+The score pass computes a quarter of its exponentials on the FMA pipe
+(`exp2_quartic2` in score_kernel.cu, packed f32x2 steps): 2^x = 2^n 2^f
+with n = round(x) and a
 quartic for 2^f on [-1/2, 1/2]. This test reads the quartic's coefficients
 from the kernel source and evaluates the same steps in fp32 (each Horner
 step rounded once, as a fused multiply-add rounds) against the exact 2^x:
 the relative error stays within the bound the kernel's comment states. It
 also re-derives the coefficients: they are the minimax fit of the relative
 error (Remez exchange, degree 4 on [-1/2, 1/2], in fp64), rounded to fp32.
+
+The attention's softmax takes a quarter of its exponentials from a cubic
+(`exp2_cubic2` in attn_fwd.cu, packed f32x2 steps); the same checks pin
+it against the degree-3 fit and its stated 7.5e-5 bound.
 """
 import os
 import re
@@ -16,30 +21,45 @@ import numpy as np
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "..", "rolling_kv_cache_b200", "csrc", "score_kernel.cu")
+ATTN_SRC = os.path.join(HERE, "..", "rolling_kv_cache_b200", "csrc", "attn_fwd.cu")
+
+
+def _packed_coefficients(src, func):
+    """Coefficients of a packed Horner polynomial `func` (highest degree
+    first), as the source spells them: every make_float2(a, a) from the
+    first `q =` step up to the return."""
+    text = open(src).read()
+    body = text[text.index(func):]
+    body = body[body.index("float2 q ="):body.index("return")]
+    vals = re.findall(r"make_float2\(([0-9.eE+-]+)f, ([0-9.eE+-]+)f\)", body)
+    assert all(a == b for a, b in vals)          # both lanes carry the same constant
+    return [np.float32(float(a)) for a, _ in vals]
 
 
 def _coefficients():
-    text = open(SRC).read()
-    body = text[text.index("float exp2_fma(float x)"):]
-    body = body[:body.index("\n}\n")]
-    lead = re.search(r"float p = ([0-9.eE+-]+)f;", body).group(1)
-    rest = re.findall(r"p = fmaf\(p, f, ([0-9.eE+-]+)f\);", body)
-    return [np.float32(float(c)) for c in [lead] + rest]   # highest degree first
+    return _packed_coefficients(SRC, "float2 exp2_quartic2(float2 x)")
 
 
-def _exp2_fma(x):
-    """The kernel's steps, vectorised, in fp32."""
+def _packed_exp2(x, coeffs):
+    """The packed exponential's steps in fp32, one lane at a time (a packed
+    f32x2 instruction rounds each lane as its scalar form does): clamp at
+    -126, t = x + 1.5 * 2^23, n = t - 1.5 * 2^23, f = fma(n, -1, x),
+    Horner in f, then t's low bits shifted into the exponent field."""
     x = np.maximum(np.asarray(x, dtype=np.float32), np.float32(-126.0))
     magic = np.float32(12582912.0)
     t = (x + magic).astype(np.float32)
-    f = (x - (t - magic).astype(np.float32)).astype(np.float32)
-    c = _coefficients()
-    p = np.full_like(f, c[0])
-    for ck in c[1:]:
-        p = (p.astype(np.float64) * f.astype(np.float64) + np.float64(ck)).astype(np.float32)
-    n = (t.view(np.int32).astype(np.int64) - 0x4B400000).astype(np.int64)
-    bits = (p.view(np.uint32).astype(np.int64) + (n << 23)) & 0xFFFFFFFF
+    n = (t - magic).astype(np.float32)
+    f = (n.astype(np.float64) * -1.0 + x.astype(np.float64)).astype(np.float32)   # one rounding
+    q = np.full_like(f, coeffs[0])
+    for ck in coeffs[1:]:
+        q = (q.astype(np.float64) * f.astype(np.float64) + np.float64(ck)).astype(np.float32)
+    bits = (q.view(np.uint32).astype(np.int64) + (t.view(np.uint32).astype(np.int64) << 23)) & 0xFFFFFFFF
     return bits.astype(np.uint32).view(np.float32)
+
+
+def _exp2_fma(x):
+    """The score pass's steps, vectorised, in fp32."""
+    return _packed_exp2(x, _coefficients())
 
 
 def test_exp2_fma_coefficients_present():
@@ -101,5 +121,35 @@ def test_exp2_fma_coefficients_are_the_minimax_fit():
     src = np.array(_coefficients()[::-1], dtype=np.float32)   # lowest degree first
     fit = c.astype(np.float32)
     # each coefficient is the fp64 minimax coefficient rounded to fp32 (within one fp32 ulp)
+    ulp = np.spacing(np.abs(fit))
+    assert np.all(np.abs(src.astype(np.float64) - fit.astype(np.float64)) <= ulp), (src, fit)
+
+
+def _cubic_coefficients():
+    return _packed_coefficients(ATTN_SRC, "float2 exp2_cubic2(float2 x)")
+
+
+def _exp2_cubic2(x):
+    return _packed_exp2(x, _cubic_coefficients())
+
+
+def test_attention_cubic_relative_error():
+    assert len(_cubic_coefficients()) == 4
+    # the softmax's arguments: s c - m c, at most the rescale threshold (8) above 0
+    x = np.concatenate([np.linspace(-125.0, 8.0, 400001, dtype=np.float32),
+                        np.linspace(-1.0, 1.0, 200001, dtype=np.float32)])
+    got = _exp2_cubic2(x).astype(np.float64)
+    want = np.exp2(x.astype(np.float64))
+    rel = np.abs(got - want) / want
+    assert rel.max() <= 7.5e-5 * 1.02, rel.max()
+    tiny = _exp2_cubic2(np.array([-np.inf, -1000.0, -126.7], dtype=np.float32)).astype(np.float64)
+    assert np.all((tiny >= 0.0) & (tiny <= 2.0 ** -125))
+
+
+def test_attention_cubic_is_the_minimax_fit():
+    c, E = _remez_relative(deg=3)
+    assert 7.4e-5 < E < 7.6e-5
+    src = np.array(_cubic_coefficients()[::-1], dtype=np.float32)   # lowest degree first
+    fit = c.astype(np.float32)
     ulp = np.spacing(np.abs(fit))
     assert np.all(np.abs(src.astype(np.float64) - fit.astype(np.float64)) <= ulp), (src, fit)
