@@ -8,6 +8,10 @@
 // selected logical indices in index order, taking every score above the
 // threshold and the lowest-index ties at it. Output is ascending; missing
 // entries (fewer candidates than C) are -1.
+// A lone CTA runs on latency, not bandwidth: the gather keeps eight loads in
+// flight per thread, and the order keys stay in shared memory for the passes
+// and the compaction (up to kTopcSmemKeys of them; a larger candidate set
+// reads its keys back from the logical-order scores in global memory).
 // The scores of one step share their top bytes, so a warp adds the count of
 // its lanes that fall in the first valid lane's bin with one atomic (the
 // rest add their own); one warp finds the threshold digit by a shuffle scan
@@ -23,6 +27,8 @@ namespace rc {
 namespace {
 
 constexpr int kTopcThreads = 1024;
+constexpr int kTopcSmemKeys = 49152;  // 192 KB of order keys
+constexpr int kTopcGather = 8;        // gather loads in flight per thread
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t b = __float_as_uint(f);
@@ -57,7 +63,8 @@ __device__ __forceinline__ long long block_exclusive_scan(long long v, long long
   return before;
 }
 
-__global__ void __launch_bounds__(kTopcThreads) topc_kernel(const __grid_constant__ TopCParams p) {
+__global__ void __launch_bounds__(kTopcThreads) topc_kernel(const __grid_constant__ TopCParams p, int keys_in_smem) {
+  extern __shared__ uint32_t skey[];  // [n] order keys, when keys_in_smem
   __shared__ int hist[256];
   __shared__ long long warp_tot[32];
   __shared__ uint32_t sh_prefix, sh_mask;
@@ -65,11 +72,27 @@ __global__ void __launch_bounds__(kTopcThreads) topc_kernel(const __grid_constan
   const int n = p.n_cand_frames * p.F;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float* lg = p.scores_out;
-  for (int i = threadIdx.x; i < n; i += kTopcThreads) {
-    const int fi = i / p.F, t = i - fi * p.F;
-    lg[i] = p.score_phys[(size_t)p.cand_slot[fi] * p.F + t];
+  for (int b = threadIdx.x; b < n; b += kTopcGather * kTopcThreads) {
+    float v[kTopcGather];
+#pragma unroll
+    for (int u = 0; u < kTopcGather; ++u) {
+      const int i = b + u * kTopcThreads;
+      if (i < n) {
+        const int fi = i / p.F, t = i - fi * p.F;
+        v[u] = p.score_phys[(size_t)p.cand_slot[fi] * p.F + t];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kTopcGather; ++u) {
+      const int i = b + u * kTopcThreads;
+      if (i < n) {
+        lg[i] = v[u];
+        if (keys_in_smem) skey[i] = order_key(v[u]);
+      }
+    }
   }
   __syncthreads();
+  auto key_at = [&](int i) -> uint32_t { return keys_in_smem ? skey[i] : order_key(lg[i]); };
   if (!p.topc || p.C <= 0) return;
   const int take = min(p.C, n);
   if (threadIdx.x == 0) {
@@ -88,7 +111,7 @@ __global__ void __launch_bounds__(kTopcThreads) topc_kernel(const __grid_constan
         const int i = b + lane;
         int digit = -1;
         if (i < n) {
-          const uint32_t key = order_key(lg[i]);
+          const uint32_t key = key_at(i);
           if ((key & mask) == prefix) digit = (int)((key >> shift) & 255u);
         }
         const uint32_t valid = __ballot_sync(0xffffffffu, digit >= 0);
@@ -140,7 +163,7 @@ __global__ void __launch_bounds__(kTopcThreads) topc_kernel(const __grid_constan
     const int i0 = min(n, threadIdx.x * per), i1 = min(n, i0 + per);
     int gt = 0, eq = 0;
     for (int i = i0; i < i1; ++i) {
-      const uint32_t key = order_key(lg[i]);
+      const uint32_t key = key_at(i);
       gt += key > thr;
       eq += key == thr;
     }
@@ -150,7 +173,7 @@ __global__ void __launch_bounds__(kTopcThreads) topc_kernel(const __grid_constan
     int pos = gt_before + min(eq_before, k_eq);
     int eq_seen = eq_before;
     for (int i = i0; i < i1; ++i) {
-      const uint32_t key = order_key(lg[i]);
+      const uint32_t key = key_at(i);
       bool sel = key > thr;
       if (key == thr) sel = eq_seen++ < k_eq;
       if (sel) {
@@ -189,7 +212,17 @@ cudaError_t launch_watchdog_selftest(int* status, unsigned limit_us, cudaStream_
 }
 
 cudaError_t launch_topc(const TopCParams& p, cudaStream_t s) {
-  topc_kernel<<<1, kTopcThreads, 0, s>>>(p);
+  static PerDevice attr_set;
+  int done = 0;
+  cudaError_t e = attr_set.get(&done, [](int, int* x) {
+    *x = 1;
+    return cudaFuncSetAttribute(topc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kTopcSmemKeys * (int)sizeof(uint32_t));
+  });
+  if (e != cudaSuccess) return e;
+  const long long n = (long long)p.n_cand_frames * p.F;
+  const int in_smem = n <= kTopcSmemKeys ? 1 : 0;
+  topc_kernel<<<1, kTopcThreads, in_smem ? (size_t)n * sizeof(uint32_t) : 0, s>>>(p, in_smem);
   return cudaGetLastError();
 }
 
