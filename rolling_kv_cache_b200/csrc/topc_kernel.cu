@@ -29,6 +29,7 @@ namespace {
 constexpr int kTopcThreads = 1024;
 constexpr int kTopcSmemKeys = 49152;  // 192 KB of order keys
 constexpr int kTopcGather = 8;        // gather loads in flight per thread
+static_assert(kTopcThreads == 1024, "the histogram sum maps 1024 threads onto 256 bins x 4 warp groups");
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t b = __float_as_uint(f);
@@ -66,20 +67,28 @@ __device__ __forceinline__ long long block_exclusive_scan(long long v, long long
 __global__ void __launch_bounds__(kTopcThreads) topc_kernel(const __grid_constant__ TopCParams p, int keys_in_smem) {
   extern __shared__ uint32_t skey[];  // [n] order keys, when keys_in_smem
   __shared__ int hist[256];
+  __shared__ int whist[kTopcThreads / 32][257];  // per-warp histograms (padded row: no bank conflicts in the sum)
   __shared__ long long warp_tot[32];
   __shared__ uint32_t sh_prefix, sh_mask;
   __shared__ int sh_k;
   const int n = p.n_cand_frames * p.F;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float* lg = p.scores_out;
+  // this thread's candidates i = threadIdx.x + m kTopcThreads, as (frame fi,
+  // token t) advanced by a fixed step instead of a division per element
+  const int step_f = kTopcThreads / p.F, step_t = kTopcThreads - step_f * p.F;
+  int fi = threadIdx.x / p.F, t = threadIdx.x - fi * p.F;
   for (int b = threadIdx.x; b < n; b += kTopcGather * kTopcThreads) {
     float v[kTopcGather];
 #pragma unroll
     for (int u = 0; u < kTopcGather; ++u) {
       const int i = b + u * kTopcThreads;
-      if (i < n) {
-        const int fi = i / p.F, t = i - fi * p.F;
-        v[u] = p.score_phys[(size_t)p.cand_slot[fi] * p.F + t];
+      if (i < n) v[u] = p.score_phys[(size_t)p.cand_slot[fi] * p.F + t];
+      fi += step_f;
+      t += step_t;
+      if (t >= p.F) {
+        t -= p.F;
+        ++fi;
       }
     }
 #pragma unroll
@@ -103,8 +112,10 @@ __global__ void __launch_bounds__(kTopcThreads) topc_kernel(const __grid_constan
   __syncthreads();
   if (take > 0) {
     for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = threadIdx.x; i < 256; i += kTopcThreads) hist[i] = 0;
-      __syncthreads();
+      // each warp counts into its own histogram (no contention between warps
+      // on the few bins the scores of one step share); summed below
+      for (int i = lane; i < 256; i += 32) whist[warp][i] = 0;
+      __syncwarp();
       const uint32_t prefix = sh_prefix, mask = sh_mask;
       // whole warps step together (b is warp-uniform) so the votes see every lane
       for (int b = warp * 32; b < n; b += kTopcThreads) {
@@ -119,8 +130,18 @@ __global__ void __launch_bounds__(kTopcThreads) topc_kernel(const __grid_constan
         const int src = __ffs(valid) - 1;
         const int lead = __shfl_sync(0xffffffffu, digit, src);
         const uint32_t same = __ballot_sync(0xffffffffu, digit == lead);
-        if (lane == src) atomicAdd(&hist[lead], __popc(same));
-        else if (digit >= 0 && digit != lead) atomicAdd(&hist[digit], 1);
+        if (lane == src) atomicAdd(&whist[warp][lead], __popc(same));
+        else if (digit >= 0 && digit != lead) atomicAdd(&whist[warp][digit], 1);
+      }
+      __syncthreads();
+      {  // bin t / 4 summed over warps 8 (t % 4) .. 8 (t % 4) + 7, then over the 4 threads
+        const int bin = threadIdx.x >> 2, w0 = (threadIdx.x & 3) * 8;
+        int c = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) c += whist[w0 + w][bin];
+        c += __shfl_xor_sync(0xffffffffu, c, 1);
+        c += __shfl_xor_sync(0xffffffffu, c, 2);
+        if ((threadIdx.x & 3) == 0) hist[bin] = c;
       }
       __syncthreads();
       if (warp == 0) {
