@@ -225,14 +225,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     ptx::tma_prefetch_desc(&p.tm_v);
     int nq = 0, g = 0;
     int nk[2] = {0, 0}, nv[2] = {0, 0};  // loads issued per stage
+    // K/V tiles are read by every query pair of their head (19 CTAs walking
+    // them at about the same time): keep them in L2; Q is read by one CTA
+    const uint64_t pol_q = ptx::l2_policy(false), pol_kv = ptx::l2_policy(true);
     bool ok = true;
     while (ok && sc.next(jb)) {
       if (nq > 0 && !ptx::mbar_wait(&bar_qe, (nq - 1) & 1, abort, p.status, RC_ETIMEOUT)) break;
       ptx::mbar_arrive_expect_tx(&bar_q, (jb.has1 ? 2 : 1) * L::kTile);
       for (int i = 0; i < (jb.has1 ? 2 : 1); ++i)
         for (int j = 0; j < L::kSub; ++j)
-          ptx::tma_load_3d(&p.tm_q, &bar_q, base + L::kQ + i * L::kTile + j * kSubTileBytes, 64 * j,
-                           jb.q0 + i * kTileRows, jb.h);
+          ptx::tma_load_3d_hint(&p.tm_q, &bar_q, base + L::kQ + i * L::kTile + j * kSubTileBytes, 64 * j,
+                                jb.q0 + i * kTileRows, jb.h, pol_q);
       ++nq;
       TileWalker wk{p.seg, p.n_segs, jb.rq_hi};
       wk.seek(jb.kv_lo);
@@ -243,14 +246,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         if (g >= 2 && !ptx::mbar_wait(&bar_ke[st], free_par, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
         ptx::mbar_arrive_expect_tx(&bar_kf[st], L::kTile);
         for (int k = 0; k < L::kSub; ++k)
-          ptx::tma_load_3d(&p.tm_k, &bar_kf[st], base + L::kK + st * L::kTile + k * kSubTileBytes, 0,
-                           t.tok, jb.h * L::kSub + k);
+          ptx::tma_load_3d_hint(&p.tm_k, &bar_kf[st], base + L::kK + st * L::kTile + k * kSubTileBytes,
+                                0, t.tok, jb.h * L::kSub + k, pol_kv);
         nk[st]++;
         if (g >= 2 && !ptx::mbar_wait(&bar_ve[st], free_par, abort, p.status, RC_ETIMEOUT)) { ok = false; break; }
         ptx::mbar_arrive_expect_tx(&bar_vf[st], L::kTile);
         for (int k = 0; k < L::kSub; ++k)
-          ptx::tma_load_3d(&p.tm_v, &bar_vf[st], base + L::kV + st * L::kTile + k * kSubTileBytes, 0,
-                           t.tok, jb.h * L::kSub + k);
+          ptx::tma_load_3d_hint(&p.tm_v, &bar_vf[st], base + L::kV + st * L::kTile + k * kSubTileBytes,
+                                0, t.tok, jb.h * L::kSub + k, pol_kv);
         nv[st]++;
       }
     }
