@@ -225,8 +225,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     ptx::tma_prefetch_desc(&p.tm_v);
     int nq = 0, g = 0;
     int nk[2] = {0, 0}, nv[2] = {0, 0};  // loads issued per stage
-    // K/V tiles are read by every query pair of their head (19 CTAs walking
-    // them at about the same time): keep them in L2; Q is read by one CTA
+    // K/V tiles are read by every query pair of their head, whose CTAs walk
+    // them at about the same time: keep them in L2; Q is read by one CTA
     const uint64_t pol_q = ptx::l2_policy(false), pol_kv = ptx::l2_policy(true);
     bool ok = true;
     while (ok && sc.next(jb)) {
