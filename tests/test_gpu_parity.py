@@ -91,12 +91,13 @@ def test_multi_tile_ragged(mask_block):
     r.close()
 
 
-@pytest.mark.parametrize("mask_block", [1, 3])
-def test_stream_k_split_units(mask_block):
+@pytest.mark.parametrize("mask_block,d", [(1, 128), (3, 128), (1, 64)])
+def test_stream_k_split_units(mask_block, d):
     # 64 heads x 3 query pairs = 192 (head, pair) units > 148 SMs: the
     # persistent schedule splits units between CTAs and the combine kernel
-    # merges their partial rows. 240-token frames keep tiles ragged.
-    w = rc_synth.Workload(name="streamk", workload_id=13, layers=1, heads=64, head_dim=128, grid_h=12,
+    # merges their partial rows (and drops their L2 lines, four threads to a
+    # line at d = 64, two at d = 128). 240-token frames keep tiles ragged.
+    w = rc_synth.Workload(name="streamk", workload_id=13, layers=1, heads=64, head_dim=d, grid_h=12,
                           grid_w=20, chunk_frames=3, sink_frames=1, window_frames=6,
                           policy=rc_synth.POLICY_SLIDING, chunks=4, mask_block_frames=mask_block)
     r = Runner(w)
