@@ -207,6 +207,21 @@ def test_infinity_rope_small_with_scores(d):
     r.close()
 
 
+@pytest.mark.parametrize("C", [2, 50])
+def test_topc_small_candidate_sets(C):
+    # 3-token frames: 3 to 45 candidates, so several of the top-C cluster's
+    # eight slices are empty or hold a few keys, and C falls below and above
+    # the candidate count
+    w = W["infinity_rope"].replace(heads=1, head_dim=64, grid_h=1, grid_w=3, chunks=10, cut_chunks=(6,),
+                                   topc=C)
+    r = Runner(w)
+    for c, p, g0, cut in rc_synth.stream_schedule(w):
+        r.step(c, p, cut, scores=True)
+        ref, _ = r.check_float(scores=True)
+        _topc_checks(w, r, ref)
+    r.close()
+
+
 def test_inplace_rerotation_bitexact():
     # Sliding with a sink time shift: the sink is re-rotated in place by delta.
     w = W["tiny"].replace(heads=2, head_dim=128, grid_h=4, grid_w=8, sink_frames=2, chunks=6)
