@@ -5,7 +5,8 @@ raises AssertionError on a mismatch, so the same check runs against the real
 oracle (tests/test_oracle_*.py) and against copies of it with a plausible
 mistake planted (tests/test_oracle_mutations.py), which it must reject.
 Nothing here reuses the oracle's formulas: RoPE is recomputed with complex
-numbers, attention with scalar Python loops, top-C by exhaustive search.
+numbers, attention with scalar Python loops, top-C by exhaustive search,
+token scores as the gradient of the summed log-sum-exp (torch autograd).
 """
 from __future__ import annotations
 
@@ -211,3 +212,30 @@ def check_topc_bruteforce(top_c_fn, seed=0):
                 winners.append(sorted(int(idx[a]) for a in sub))
         assert len(winners) == 1
         assert got == winners[0], (scores, idx, C, got, winners)
+
+
+def check_column_scores_autograd(column_scores_fn, seed=0):
+    """Token scores as a derivative: for lse_q = log sum_j exp(s_qj + b_j),
+    d lse_q / d b_j is the probability p_qj, so the gradient of the summed
+    log-sum-exp over every head and query with respect to a per-key logit
+    bias b is each key's received attention mass. torch autograd computes it
+    from the logits alone; the oracle's function gets the probabilities and a
+    candidate subset of the key columns, whose scores it must return in the
+    subset's order."""
+    import torch
+    rng = np.random.default_rng(seed)
+    for H, nq, nk, d in ((1, 3, 5, 4), (3, 7, 19, 8), (4, 12, 40, 16)):
+        q = torch.from_numpy(rng.standard_normal((H, nq, d)))
+        k = torch.from_numpy(rng.standard_normal((H, nk, d)))
+        vis = rng.random((nq, nk)) < 0.6
+        vis[:, int(rng.integers(nk))] = True
+        logits = torch.where(torch.from_numpy(vis)[None], q @ k.transpose(1, 2) / math.sqrt(d),
+                             torch.tensor(-math.inf, dtype=torch.float64))
+        b = torch.zeros(nk, dtype=torch.float64, requires_grad=True)
+        torch.logsumexp(logits + b, dim=2).sum().backward()
+        mass = b.grad.numpy()
+        p_per_head = [torch.softmax(logits[h], dim=1).numpy() for h in range(H)]
+        cols = np.sort(rng.choice(nk, size=max(1, nk // 2), replace=False))
+        got = np.asarray(column_scores_fn(p_per_head, cols))
+        assert got.shape == cols.shape, (got.shape, cols.shape)
+        assert np.allclose(got, mass[cols], rtol=0, atol=1e-12), (got, mass[cols])

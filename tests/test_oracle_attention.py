@@ -75,6 +75,10 @@ def test_column_scores_total_mass():
     assert abs(total - 3 * 5) < 1e-12
 
 
+def test_column_scores_are_the_logit_bias_gradient():
+    pins.check_column_scores_autograd(column_scores)
+
+
 TINY = rc_synth.Workload(name="brute", workload_id=9, layers=1, heads=2, head_dim=8,
                          grid_h=2, grid_w=2, chunk_frames=2, sink_frames=1,
                          window_frames=100, policy=rc_synth.POLICY_SLIDING, chunks=4)

@@ -6,6 +6,8 @@ nothing here touches the library or a GPU.
 import numpy as np
 import pytest
 
+import rc_synth
+
 import oracle.attention as oatt
 import oracle.policy as opol
 import oracle.rope as orope
@@ -225,3 +227,56 @@ def test_memrope_pins_reject_zero_initialised_memories(monkeypatch):
         return orig_step(self, frame_start, n_frames)
     monkeypatch.setattr(omr.MemRopeOracle, "step", step)
     assert _rejected((tmr.test_hand_computed_memories, ()), (tmr.test_ema_closed_form_and_extremes, (0.3,)))
+
+
+# ---- token scores and the in-chunk mask
+
+def _scores_per_query(p_per_head, cols):
+    # the mass each query gives the candidates, not the mass each candidate gets
+    return sum(p[:, cols].sum(axis=1) for p in p_per_head)
+
+
+def _scores_mean_over_heads(p_per_head, cols):
+    return oatt.column_scores(p_per_head, cols) / len(p_per_head)
+
+
+def _scores_first_head_only(p_per_head, cols):
+    return oatt.column_scores(p_per_head[:1], cols)
+
+
+def _scores_shifted_column(p_per_head, cols):
+    n = p_per_head[0].shape[1]
+    return oatt.column_scores(p_per_head, (np.asarray(cols) + 1) % n)
+
+
+@pytest.mark.parametrize("fn", [_scores_per_query, _scores_mean_over_heads, _scores_first_head_only,
+                                _scores_shifted_column])
+def test_column_scores_pin_rejects(fn):
+    with pytest.raises(AssertionError):
+        pins.check_column_scores_autograd(fn)
+
+
+import oracle.stream as ostream
+import test_oracle_attention as tatt
+
+
+def _vis_strict(query_rank, key_rank, mask_block_frames=1):
+    # a frame no longer sees its own keys
+    qr = np.asarray(query_rank)[:, None] // mask_block_frames
+    kr = np.asarray(key_rank)[None, :]
+    return (kr < 0) | ((kr // mask_block_frames) < qr)
+
+
+def _vis_unblocked_keys(query_rank, key_rank, mask_block_frames=1):
+    # the block size applied to the query side only
+    qr = np.asarray(query_rank)[:, None] // mask_block_frames
+    kr = np.asarray(key_rank)[None, :]
+    return (kr < 0) | (kr <= qr)
+
+
+@pytest.mark.parametrize("fn,mask_block", [(_vis_strict, 1), (_vis_unblocked_keys, 2)])
+def test_visibility_pins_reject(fn, mask_block, monkeypatch):
+    monkeypatch.setattr(ostream, "visibility", fn)
+    with np.errstate(invalid="ignore"):   # the strict mask leaves the first frame's rows empty
+        assert _rejected((tatt.test_window_covering_history_is_full_causal_attention,
+                          (rc_synth.POLICY_SLIDING, mask_block)))
