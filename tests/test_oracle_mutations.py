@@ -280,3 +280,15 @@ def test_visibility_pins_reject(fn, mask_block, monkeypatch):
     with np.errstate(invalid="ignore"):   # the strict mask leaves the first frame's rows empty
         assert _rejected((tatt.test_window_covering_history_is_full_causal_attention,
                           (rc_synth.POLICY_SLIDING, mask_block)))
+
+
+import test_oracle_policy as tpol
+
+
+@pytest.mark.parametrize("fn", [
+    lambda prev, new: opol.evicted_contents(new, prev),              # what arrived, not what left
+    lambda prev, new: sorted({k.content for k in prev} - {k.content for k in new})[1:],  # one lost
+])
+def test_eviction_pin_rejects(fn):
+    with pytest.raises(AssertionError):
+        tpol.check_eviction_is_the_oldest_window_frames(fn)

@@ -49,6 +49,34 @@ def test_lingbot_worked_numbers():
                                w.window_frames, w.chunk_frames, w.chunks)
 
 
+
+def check_eviction_is_the_oldest_window_frames(evicted_fn):
+    """LingBot's cache (sink + window frames) at steady state drops, per
+    chunk, the chunk's worth of oldest non-sink frames it held before: 3
+    frames = 4680 tokens at 1560-token frames, as its worked numbers say."""
+    w = rc_synth.WORKLOADS["large"]
+    B, S, W, F = w.chunk_frames, w.sink_frames, w.window_frames, w.frame_seqlen
+    pol = PolicyOracle(1, B, S, W)
+    prev, steady = None, 0
+    for c in range(w.chunks + 6):
+        kept = pol.step(c * B, B)
+        if prev is not None:
+            ev = list(evicted_fn(prev, kept))
+            older = sorted(k.content for k in prev if k.region != "sink")
+            if len(prev) == S + W:
+                assert ev == older[:B]
+                assert len(ev) * F == 4680
+                steady += 1
+            else:
+                assert ev == []
+        prev = kept
+    assert steady >= 1
+
+
+def test_evicted_contents_are_the_oldest_window_frames():
+    check_eviction_is_the_oldest_window_frames(evicted_contents)
+
+
 FRAME_POLICIES = [n for n, w in rc_synth.WORKLOADS.items()
                   if w.policy not in (rc_synth.POLICY_DEEP_FORCING, rc_synth.POLICY_RELAX_FORCING,
                                       rc_synth.POLICY_MEMROPE)]
