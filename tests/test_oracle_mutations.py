@@ -292,3 +292,16 @@ import test_oracle_policy as tpol
 def test_eviction_pin_rejects(fn):
     with pytest.raises(AssertionError):
         tpol.check_eviction_is_the_oldest_window_frames(fn)
+
+
+def _grid_column_major(frame_seqlen, grid_w):
+    # tokens walked down columns instead of along rows
+    grid_h = frame_seqlen // grid_w
+    n = np.arange(frame_seqlen)
+    return n % grid_h, n // grid_h
+
+
+def test_grid_positions_pin_rejects_column_major(monkeypatch):
+    monkeypatch.setattr(ostream, "token_grid_positions", _grid_column_major)
+    assert _rejected((tatt.test_window_covering_history_is_full_causal_attention,
+                      (rc_synth.POLICY_SLIDING, 1)))
